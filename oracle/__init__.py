@@ -1,0 +1,7 @@
+"""Float64 CPU oracle for TwoTower block attention (test infrastructure only).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline legs of
+``bench.py`` may import this package.  The CUDA library never does.
+"""
+from .oracle import attend_rows, block_attn, block_causal  # noqa: F401
+from .brute import brute_block_attn, brute_block_causal  # noqa: F401
