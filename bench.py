@@ -1,0 +1,422 @@
+"""Benchmark of TwoTower block attention on B200 through the C ABI.
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--workload ID] [--impl native|reference]
+
+One step = one decode call (the whole hot path: Q pack, context KV stream,
+QK^T, online softmax, PV, block-KV fold-in, ragged mask, epilogue, split
+combine) over one batch of the named workload (default: the decode workload
+B=8, Hq=32, Hkv=2, D=128, S=16, L=4096 with 1% peaky keys), or one
+block-causal call for workload 5.  Inputs are resident in HBM before timing;
+each timed step reads a different copy of the inputs and the copies together
+exceed twice the L2 size, so no step is served from L2.  Timing: CUDA events
+on the launching stream around K graph-launched steps, max over ranks.
+
+Prints one JSON line (rank 0).  Multi-GPU runs are replicas: every rank runs
+the same per-GPU batch on its own GPU (weak scaling, no data-path
+collective); the process group only carries the barrier and the max of the
+timings.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import tempfile
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "block-attn KV GB/s & TFLOP/s on 1 B200, % of roofline; oracle CPU time"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", type=int, default=2, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--kernel", default="auto", choices=["auto", "tcgen05", "mma_sync"])
+    ap.add_argument("--no-graph", action="store_true", help="launch steps directly instead of via CUDA graphs")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def kernel_source_hash(kind: str) -> str:
+    files = {"tcgen05": ["attn_tcgen05.cu"], "mma_sync": ["attn_mma_sync.cu"]}[kind]
+    h = hashlib.sha256()
+    for f in files + ["ptx.cuh", "walker.cuh", "problem.h", "sched.cuh"]:
+        h.update(open(os.path.join(ROOT, "two_tower_block_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kind: str, workload: int):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on the
+    current kernel source (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(p):
+        return None
+    want = kernel_source_hash(kind)
+    for line in open(p):
+        line = line.split("#", 1)[0].split()
+        if len(line) == 4 and line[0] == kind and line[1] == want and int(line[2]) == workload:
+            return float(line[3])
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+    Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                rows.append((float(parts[0]), float(parts[1]), parts[3:7]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i, v in enumerate(r) if v.lower() == "active"})
+        sm = [r[0] for r in rows]
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
+                "samples": len(rows)}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    pg = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        backend = "nccl" if args.impl == "native" else "gloo"
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+        pg = dist
+    return world, rank, local, pg
+
+
+def max_over_ranks(pg, value, device=None):
+    if pg is None:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def workload_cost(wid, inp):
+    from two_tower_block_b200.workloads import WORKLOADS, causal_cost, decode_cost
+    w = WORKLOADS[wid]
+    if w.kind == "decode":
+        return decode_cost(w.batch, w.block_size, w.num_q_heads, w.num_kv_heads, w.head_dim, inp.ctx_lens)
+    return causal_cost(w.batch, w.seq_len, w.block_size, w.num_q_heads, w.num_kv_heads, w.head_dim)
+
+
+# --------------------------------------------------------------- oracle arm --
+def oracle_sample(wid, inp, seconds):
+    """Time the float64 oracle, as it stands, on a bounded sample of the workload.
+    Returns (GB/s of algorithmic bytes, description, threads)."""
+    from oracle import block_attn, block_causal
+    from two_tower_block_b200.workloads import WORKLOADS, bf16_to_f64, causal_cost, decode_cost
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        threads = 1
+    w = WORKLOADS[wid]
+    done_bytes = 0
+    units = 0
+    t0 = time.perf_counter()
+    n = 0
+    while time.perf_counter() - t0 < seconds:
+        if w.kind == "decode":
+            b = n % w.batch
+            sl = slice(b, b + 1)
+            block_attn(bf16_to_f64(inp.q[sl]), bf16_to_f64(inp.k_ctx[sl]), bf16_to_f64(inp.v_ctx[sl]),
+                       bf16_to_f64(inp.k_blk[sl]), bf16_to_f64(inp.v_blk[sl]), inp.ctx_lens[sl])
+            done_bytes += decode_cost(1, w.block_size, w.num_q_heads, w.num_kv_heads, w.head_dim,
+                                      inp.ctx_lens[sl])["bytes"]
+            units += 1
+        else:
+            nb = w.seq_len // w.block_size
+            b = (n * 37) % nb
+            sl = slice(0, 1)
+            block_causal(bf16_to_f64(inp.q[sl]), bf16_to_f64(inp.k_ctx[sl]), bf16_to_f64(inp.v_ctx[sl]),
+                         bf16_to_f64(inp.k_blk[sl]), bf16_to_f64(inp.v_blk[sl]), w.block_size, blocks=[b])
+            L = w.block_size * b
+            done_bytes += decode_cost(1, w.block_size, w.num_q_heads, w.num_kv_heads, w.head_dim, [L])["bytes"]
+            units += 1
+        n += 1
+    el = time.perf_counter() - t0
+    what = "sequences" if w.kind == "decode" else "blocks of sequence 0"
+    return done_bytes / el / 1e9, f"{units} {what} of the workload in {el:.1f} s", threads, el
+
+
+def run_reference(args):
+    # Under torchrun only rank 0 times the oracle; the others exit without work.
+    if int(os.environ.get("RANK", "0")) != 0:
+        return 0
+    from two_tower_block_b200.workloads import WORKLOADS, make_workload
+    w = WORKLOADS[args.workload]
+    inp = make_workload(args.workload)
+    per_step = max(1.0, min(8.0, 120.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_sample(args.workload, inp, per_step / 4)
+    vals = []
+    t_all = 0.0
+    desc = ""
+    threads = 1
+    for _ in range(args.steps):
+        v, desc, threads, el = oracle_sample(args.workload, inp, per_step)
+        vals.append(v)
+        t_all += el
+    value = float(np.mean(vals))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1000 * t_all / args.steps, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": w.describe(),
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+                         "sample": f"each step: {desc}"},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------- native arm --
+def run_native(args):
+    import torch
+    world, rank, local, pg = dist_setup(args)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    from two_tower_block_b200 import ops
+    from two_tower_block_b200.workloads import WORKLOADS, make_workload
+    w = WORKLOADS[args.workload]
+    kernel = {"auto": ops.KERNEL_AUTO, "tcgen05": ops.KERNEL_TCGEN05, "mma_sync": ops.KERNEL_MMA_SYNC}[args.kernel]
+    inp = make_workload(args.workload)
+    cost = workload_cost(args.workload, inp)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+
+    def to_dev(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    base = [to_dev(inp.q), to_dev(inp.k_ctx), to_dev(inp.v_ctx), to_dev(inp.k_blk), to_dev(inp.v_blk)]
+    in_bytes = sum(t.numel() * 2 for t in base)
+    n_copies = max(1, math.ceil(2.0 * l2 / in_bytes) + 1)
+    copies = [base] + [[t.clone() for t in base] for _ in range(n_copies - 1)]
+    if w.kind == "decode":
+        lens = torch.from_numpy(inp.ctx_lens).to(dev)
+        plan = ops.Plan(w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_size, ctx_capacity=w.ctx,
+                        kernel=kernel, device=local)
+        out = torch.empty((w.batch, w.block_size, w.num_q_heads, w.head_dim), dtype=torch.float32, device=dev)
+        lse = torch.empty((w.batch, w.num_q_heads, w.block_size), dtype=torch.float32, device=dev)
+
+        def step(i):
+            c = copies[i % n_copies]
+            plan.block_attn(c[0], c[1], c[2], c[3], c[4], lens, out=out, lse=lse)
+    else:
+        plan = ops.Plan(w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_size, seq_len=w.seq_len,
+                        kernel=kernel, device=local)
+        out = torch.empty((w.batch, w.seq_len, w.num_q_heads, w.head_dim), dtype=torch.float32, device=dev)
+        lse = torch.empty((w.batch, w.num_q_heads, w.seq_len), dtype=torch.float32, device=dev)
+
+        def step(i):
+            c = copies[i % n_copies]
+            plan.block_attn_block_causal(c[0], c[1], c[2], c[3], c[4], out=out, lse=lse)
+
+    info = plan.info()
+    kname = {1: "tcgen05", 2: "mma_sync"}[info.kernel]
+    stream = torch.cuda.current_stream()
+    for i in range(max(3, args.warmup)):
+        step(i)
+    plan.check()
+
+    graphs = None
+    if not args.no_graph:
+        graphs = []
+        for i in range(n_copies):
+            gph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gph):
+                step(i)
+            graphs.append(gph)
+        for i in range(n_copies):
+            graphs[i].replay()
+        torch.cuda.synchronize()
+
+    clocks = ClockSampler(local)
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)  # let the sampler attach before the timed region
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        if graphs:
+            graphs[i % n_copies].replay()
+        else:
+            step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if pg:
+        pg.barrier()
+    ms_total = e0.elapsed_time(e1)
+    # per-kernel durations of the same steps, from events the library records on the launching stream
+    plan.profile(True)
+    for i in range(args.steps):
+        step(i)
+    torch.cuda.synchronize()
+    n_k, ms_k = plan.profile_read(0)
+    n_c, ms_c = plan.profile_read(1) if info.num_ctas > 1 else (0, 0.0)
+    plan.profile(False)
+    ck = clocks.stop()
+    plan.check()
+    ms_total = max_over_ranks(pg, ms_total, dev)
+    ms_step = ms_total / args.steps
+    launches_per_step = 1 + (1 if info.num_ctas > 1 else 0)
+
+    # ---- end to end through the host-buffer entry (decode workloads) ----
+    e2e = None
+    if w.kind == "decode" and not args.no_e2e:
+        hplan = ops.Plan(w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_size, ctx_capacity=w.ctx,
+                         kernel=kernel, host_io=True, device=local)
+
+        def pinned(bits):
+            return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).pin_memory()
+        hin = [pinned(inp.q), pinned(inp.k_ctx), pinned(inp.v_ctx), pinned(inp.k_blk), pinned(inp.v_blk),
+               torch.from_numpy(inp.ctx_lens).pin_memory()]
+        hout = torch.empty(tuple(out.shape), dtype=torch.float32).pin_memory()
+        hlse = torch.empty(tuple(lse.shape), dtype=torch.float32).pin_memory()
+        for _ in range(2):
+            hplan.block_attn_host(*hin, hout, hlse)
+        torch.cuda.synchronize()
+        n_e2e = max(3, min(args.steps, 20))
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(n_e2e):
+            hplan.block_attn_host(*hin, hout, hlse)
+        a1.record(stream)
+        torch.cuda.synchronize()
+        hplan.check()
+        ms_e2e = max_over_ranks(pg, a0.elapsed_time(a1) / n_e2e, dev)
+        h2d = sum(t.numel() * t.element_size() for t in hin)
+        d2h = hout.numel() * 4 + hlse.numel() * 4
+        e2e = {"value": round(world * cost["bytes"] / (ms_e2e * 1e-3) / 1e9, 3), "unit": "GB/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": round(ms_e2e, 4),
+               "steps": n_e2e}
+
+    # ---- oracle CPU baseline (rank 0, N = 1 only) ----
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        v, desc, threads, el = oracle_sample(args.workload, inp, args.cpu_seconds)
+        cpu = {"value": round(v, 5), "unit": "GB/s", "cores": threads, "kind": "oracle",
+               "sample": desc + f"; host has {os.cpu_count()} logical CPUs"}
+
+    if rank != 0:
+        return 0
+    peaks = load_peaks()
+    value = world * cost["bytes"] / (ms_step * 1e-3) / 1e9
+    tflops = world * cost["flops"] / (ms_step * 1e-3) / 1e12
+    k_ms = ms_k / max(n_k, 1)
+    achieved = cost["bytes"] / (k_ms * 1e-3) / 1e9
+    bound = "hbm" if w.kind == "decode" else "tensor"
+    if bound == "hbm":
+        roof = {"bound": "hbm", "achieved": round(achieved, 2), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": recorded_traffic(kname, args.workload),
+                "kernel": f"attn_{kname}", "kernel_ms": round(k_ms, 5),
+                "peak_source": peaks["source"] + " (hbm_gbs, copy)"}
+    else:
+        ach_t = cost["flops"] / (k_ms * 1e-3) / 1e12
+        pk = peaks["bf16_tflops_sustained"] or peaks["bf16_tflops"]
+        roof = {"bound": "tensor", "achieved": round(ach_t, 2), "peak": pk, "unit": "TFLOP/s",
+                "frac": round(ach_t / pk, 4), "traffic": recorded_traffic(kname, args.workload),
+                "kernel": f"attn_{kname}", "kernel_ms": round(k_ms, 5),
+                "peak_source": peaks["source"] + " (bf16_tflops_sustained, cuBLAS)"}
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(w.describe(), parallelism=f"replicas{world}",
+                       l2="inputs rotate over %d copies (%.0f MB) > 2x L2 (%d MB)" % (
+                           n_copies, n_copies * in_bytes / 1e6, l2 // 2**20),
+                       timing="graph replay" if graphs else "direct launches"),
+        "tflops": round(tflops, 2),
+        "tensor_frac": round(tflops / peaks["bf16_tflops"], 4),
+        "roofline": roof,
+        "combine_kernel_ms": round(ms_c / max(n_c, 1), 5) if n_c else None,
+        "gpu_launches": launches_per_step * args.steps,
+        "kernel": kname,
+        "num_ctas": info.num_ctas,
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+        "clocks": ck,
+    }
+    print(json.dumps(line), flush=True)
+    if pg:
+        pg.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_native(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

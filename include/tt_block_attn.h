@@ -1,0 +1,189 @@
+/*
+ * tt_block_attn.h -- C ABI of the TwoTower layer-aligned block attention on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The operation (paperfeed.app review of arXiv 2606.26493, "Nemotron-Labs-
+ * TwoTower", section "The idea: freeze the reader, train the writer"): at
+ * every attention layer i of the denoiser tower, the S noisy tokens of the
+ * current block b form the queries Q_b^(i); the keys and values are the
+ * frozen context tower's layer-i KV cache over every committed token,
+ * followed by the denoiser's own KV for the block.  The cache is fully
+ * visible (only the context tower itself is causal), attention inside the
+ * block is bidirectional ("masked tokens can look at each other"), and one
+ * softmax runs over the concatenation.  The page's equation was lost in
+ * extraction; the single joint softmax is the reading of its prose.
+ *
+ * For sequence n, query head j (KV head h = j / g, g = Hq / Hkv) and block
+ * row t:
+ *     keys  = { k_ctx[n,h,l] : 0 <= l < L_n }  ++  { k_blk[n,u,h] : 0 <= u < S }
+ *     s_k   = scale * <q[n,t,j], k>
+ *     out   = sum_k exp(s_k - m) v_k / sum_k exp(s_k - m),  m = max_k s_k
+ *     lse   = m + ln sum_k exp(s_k - m)
+ *
+ * The block-causal entry point is the training / prefill form (same review,
+ * section "Training and sampling": block b conditions on the frozen caches
+ * c_{<b} and on itself): block b of a length-N sequence attends to context
+ * positions [0, S*b) and to its own block positions [S*b, S*b+S).
+ *
+ * Conventions shared by every entry point
+ *   - Tensors are dense, row-major, device memory owned by the caller.
+ *     q, k_*, v_* are bf16; out and lse are fp32; ctx_lens is int32.
+ *     Every tensor pointer must be 16-byte aligned.
+ *   - Calls are asynchronous and ordered on `stream`; none synchronises the
+ *     host except tt_block_attn_check and tt_block_attn_profile_read.
+ *   - A plan may be used by one stream at a time (it owns scratch memory).
+ *   - Errors the host can see are returned synchronously.  Errors only the
+ *     device can see (ctx_lens out of range, a pipeline wait that timed out)
+ *     set the plan's device error word; the call's output is then
+ *     unspecified and tt_block_attn_check reports the error.  No kernel traps.
+ *   - Thread safety: distinct plans may be used from distinct threads.
+ */
+#ifndef TT_BLOCK_ATTN_H
+#define TT_BLOCK_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define TT_API __attribute__((visibility("default")))
+#else
+#define TT_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;                     /* same type as cudaStream_t */
+typedef struct CUstream_st* tt_stream_t;
+
+typedef enum {
+  TT_OK = 0,
+  TT_ERR_INVALID_ARG = 1,   /* null / misaligned pointer, bad descriptor or size     */
+  TT_ERR_UNSUPPORTED = 2,   /* valid but not implemented (e.g. head_dim 96)          */
+  TT_ERR_CUDA = 3,          /* a CUDA runtime call or a kernel launch failed         */
+  TT_ERR_DEVICE_ARG = 4,    /* seen on the device: ctx_lens[n] < 0 or > capacity     */
+  TT_ERR_TIMEOUT = 5        /* seen on the device: a pipeline wait ran out its limit */
+} tt_status_t;
+
+typedef enum {
+  TT_KERNEL_AUTO = 0,       /* the tcgen05 kernel                                    */
+  TT_KERNEL_TCGEN05 = 1,    /* warp-specialised TMA + tcgen05.mma + TMEM kernel      */
+  TT_KERNEL_MMA_SYNC = 2    /* warp-level mma.sync baseline kernel                   */
+} tt_kernel_t;
+
+#define TT_PLAN_HOST_IO 1   /* flags: allocate device staging for tt_block_attn_host */
+
+typedef struct {
+  int batch;          /* B >= 0 (B = 0 makes every call a no-op)                    */
+  int num_q_heads;    /* Hq >= 1                                                     */
+  int num_kv_heads;   /* Hkv >= 1, Hq % Hkv == 0; query head j reads KV head j/(Hq/Hkv) */
+  int head_dim;       /* D: 64 or 128                                                */
+  int block_size;     /* S >= 1 with S * (Hq / Hkv) <= 256                           */
+  int ctx_capacity;   /* decode: Lcap >= 0, the token stride of k_ctx / v_ctx        */
+  int seq_len;        /* block-causal: N >= 0, N % S == 0 (0: decode-only plan)      */
+  float scale;        /* softmax scale; 0 selects 1/sqrt(head_dim)                   */
+  int kernel;         /* tt_kernel_t                                                 */
+  int num_ctas;       /* persistent grid size; 0 selects the device's SM count       */
+  int flags;          /* TT_PLAN_HOST_IO or 0                                        */
+  int wait_timeout_us;/* limit of every in-kernel wait; 0 selects 1000000 (1 s)      */
+} tt_block_attn_desc;
+
+typedef struct tt_plan_s* tt_plan_t;
+
+typedef struct {
+  int kernel;              /* tt_kernel_t actually used                               */
+  int num_ctas;            /* work ranges (persistent CTAs)                           */
+  int key_tile;            /* keys per pipeline tile                                  */
+  int rows_per_unit;       /* S * g, the packed query rows of one (sequence, KV head) */
+  size_t workspace_bytes;  /* device scratch owned by the plan                        */
+  int sm_count;
+} tt_plan_info;
+
+/* Create a plan: validates the descriptor, picks the kernel and the work split
+ * for `device`, and allocates every piece of device scratch the calls need
+ * (split partials, per-range records, the error word, optional host-IO
+ * staging).  The calls themselves never allocate.  Returns TT_ERR_INVALID_ARG
+ * for a malformed descriptor, TT_ERR_UNSUPPORTED for head_dim other than
+ * 64/128 or S*g > 256, TT_ERR_CUDA if allocation fails.  *out_plan is set only
+ * on TT_OK; release it with tt_block_attn_plan_destroy. */
+TT_API tt_status_t tt_block_attn_plan(const tt_block_attn_desc* desc, int device, tt_plan_t* out_plan);
+
+TT_API void tt_block_attn_plan_destroy(tt_plan_t plan);
+
+TT_API tt_status_t tt_block_attn_plan_get_info(tt_plan_t plan, tt_plan_info* info);
+
+/* Decode-time block attention (one denoising step of one attention layer).
+ *   q        [B, S, Hq, D]    bf16  queries of the block's S noisy tokens
+ *   k_ctx    [B, Hkv, Lcap, D] bf16 context-tower layer-i keys (rows >= L_n unread)
+ *   v_ctx    [B, Hkv, Lcap, D] bf16 context-tower layer-i values
+ *   k_blk    [B, S, Hkv, D]   bf16  the denoiser's own block keys
+ *   v_blk    [B, S, Hkv, D]   bf16  the denoiser's own block values
+ *   ctx_lens [B]              int32 committed context length L_n, 0 <= L_n <= Lcap
+ *   out      [B, S, Hq, D]    fp32  attention output
+ *   lse      [B, Hq, S]       fp32  natural-log log-sum-exp per row; may be NULL
+ * Context rows at or beyond L_n are never used, whatever they hold.  Out-of-range
+ * ctx_lens values are clamped on the device and flagged TT_ERR_DEVICE_ARG. */
+TT_API tt_status_t tt_block_attn(tt_plan_t plan, const void* q, const void* k_ctx, const void* v_ctx,
+                          const void* k_blk, const void* v_blk, const int32_t* ctx_lens,
+                          float* out, float* lse, tt_stream_t stream);
+
+/* Block-causal training / prefill form over whole sequences of length N = seq_len.
+ *   q      [B, N, Hq, D]  bf16      out [B, N, Hq, D] fp32
+ *   k_ctx  [B, Hkv, N, D] bf16 (context tower over the clean sequence), v_ctx likewise
+ *   k_blk  [B, N, Hkv, D] bf16 (denoiser over the noisy sequence),     v_blk likewise
+ *   lse    [B, Hq, N] fp32 natural log, may be NULL
+ * Block b = positions [S*b, S*b+S) attends to k_ctx positions [0, S*b) and to its
+ * own k_blk positions, bidirectionally.  Requires a plan with seq_len > 0. */
+TT_API tt_status_t tt_block_attn_block_causal(tt_plan_t plan, const void* q, const void* k_ctx,
+                                       const void* v_ctx, const void* k_blk, const void* v_blk,
+                                       float* out, float* lse, tt_stream_t stream);
+
+/* Decode from HOST buffers (same layouts as tt_block_attn, same shapes as the plan):
+ * copies the inputs into plan-owned device staging (the plan needs TT_PLAN_HOST_IO),
+ * runs tt_block_attn, and copies out (and lse, when non-NULL) back, all ordered on
+ * `stream`.  One cudaMemcpyAsync per buffer.  Host buffers should be page-locked
+ * for the copies to be asynchronous and must stay valid until the stream has
+ * been synchronised; the call itself does not synchronise. */
+TT_API tt_status_t tt_block_attn_host(tt_plan_t plan, const void* q, const void* k_ctx, const void* v_ctx,
+                               const void* k_blk, const void* v_blk, const int32_t* ctx_lens,
+                               float* out, float* lse, tt_stream_t stream);
+
+/* Synchronise `stream`, then read and clear the plan's device error word.
+ * Returns TT_OK, TT_ERR_DEVICE_ARG or TT_ERR_TIMEOUT (or TT_ERR_CUDA if the
+ * synchronisation itself failed). */
+TT_API tt_status_t tt_block_attn_check(tt_plan_t plan, tt_stream_t stream);
+
+/* Per-kernel timing hook.  While enabled, every kernel the plan launches is
+ * bracketed by two CUDA events recorded on the launching stream (up to 4096
+ * launches are kept).  tt_block_attn_profile_read synchronises on the recorded
+ * events and returns, for kernel id 0 (attention) or 1 (split combine), the
+ * number of launches and their summed duration in milliseconds, then clears
+ * the record. */
+TT_API tt_status_t tt_block_attn_profile(tt_plan_t plan, int enable);
+TT_API tt_status_t tt_block_attn_profile_read(tt_plan_t plan, int kernel_id, int* launches, double* total_ms);
+
+/* Failure-path self test: launches one CTA that waits on a shared-memory
+ * barrier nothing arrives at, using the same bounded wait as the attention
+ * kernels, with a limit of `timeout_us`.  Expected result: TT_ERR_TIMEOUT, with
+ * the device context still usable afterwards. */
+TT_API tt_status_t tt_selftest_wait_timeout(int device, int timeout_us, tt_stream_t stream);
+
+/* Host-only view of the work split (no GPU needed): for `num_units` units with
+ * tiles_per_unit[u] tiles each over `num_ctas` ranges, writes for every range c
+ * its first global tile (range_start[c], num_ctas+1 entries) and, per unit, the
+ * first and last range that touch it (unit_first[u], unit_last[u]).  The same
+ * code decides the split inside the kernels. */
+TT_API tt_status_t tt_debug_work_split(int num_units, const int* tiles_per_unit, int num_ctas,
+                                long long* range_start, int* unit_first, int* unit_last);
+
+TT_API const char* tt_status_string(tt_status_t status);
+
+/* Detail of the last host-side error on the calling thread ("" if none). */
+TT_API const char* tt_last_error_detail(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TT_BLOCK_ATTN_H */

@@ -1,0 +1,110 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every symbol the header declares, rejects malformed descriptors before
+touching a device, and its work split covers every tile exactly once."""
+import os
+import re
+
+import numpy as np
+import pytest
+
+from two_tower_block_b200 import ops
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def header_symbols():
+    src = open(os.path.join(ROOT, "include", "tt_block_attn.h")).read()
+    return sorted(set(re.findall(r"TT_API\s+[\w\s\*]*?\b(tt_\w+)\s*\(", src)))
+
+
+def test_header_symbols_are_exported():
+    L = ops.lib()
+    syms = header_symbols()
+    assert len(syms) >= 13
+    for s in syms:
+        assert hasattr(L, s), f"{s} declared in the header but not exported"
+    assert sorted(ops.EXPORTED_SYMBOLS) == syms
+
+
+def test_exported_symbols_via_nm():
+    import shutil
+    import subprocess
+    nm = shutil.which("nm")
+    if nm is None:
+        pytest.skip("nm not available")
+    out = subprocess.run([nm, "-D", "--defined-only", ops.library_path], capture_output=True, text=True).stdout
+    exported = set(re.findall(r" T (tt_\w+)", out))
+    assert set(header_symbols()) <= exported
+
+
+def test_status_strings():
+    L = ops.lib()
+    for s in range(6):
+        assert L.tt_status_string(s)
+    assert b"timed out" in L.tt_status_string(ops.TT_ERR_TIMEOUT)
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(head_dim=96), ops.TT_ERR_UNSUPPORTED),
+    (dict(num_q_heads=6, num_kv_heads=4), ops.TT_ERR_INVALID_ARG),
+    (dict(block_size=0), ops.TT_ERR_INVALID_ARG),
+    (dict(block_size=32, num_q_heads=32, num_kv_heads=2), ops.TT_ERR_UNSUPPORTED),  # S*g = 512
+    (dict(seq_len=100, block_size=16), ops.TT_ERR_INVALID_ARG),
+    (dict(batch=-1), ops.TT_ERR_INVALID_ARG),
+    (dict(scale=-1.0), ops.TT_ERR_INVALID_ARG),
+    (dict(kernel=9), ops.TT_ERR_INVALID_ARG),
+    (dict(flags=4), ops.TT_ERR_INVALID_ARG),
+])
+def test_descriptor_validation_before_device(bad, code):
+    import ctypes
+    d = dict(batch=2, num_q_heads=8, num_kv_heads=2, head_dim=128, block_size=16, ctx_capacity=64,
+             seq_len=0, scale=0.0, kernel=0, num_ctas=0, flags=0, wait_timeout_us=0)
+    d.update(bad)
+    desc = ops.Desc(**d)
+    h = ctypes.c_void_p()
+    st = ops.lib().tt_block_attn_plan(ctypes.byref(desc), 0, ctypes.byref(h))
+    assert st == code, ops.lib().tt_last_error_detail()
+    assert not h.value
+
+
+def test_null_arguments():
+    L = ops.lib()
+    assert L.tt_block_attn_plan(None, 0, None) == ops.TT_ERR_INVALID_ARG
+    assert L.tt_block_attn(None, *([None] * 9)) == ops.TT_ERR_INVALID_ARG
+    assert L.tt_block_attn_check(None, None) == ops.TT_ERR_INVALID_ARG
+    L.tt_block_attn_plan_destroy(None)  # no-op
+
+
+@pytest.mark.parametrize("tiles,C", [
+    ([3, 5, 1, 7], 4), ([1] * 17, 5), ([40], 148), ([2, 2], 7), ([33] * 16, 148),
+    (list(np.random.default_rng(0).integers(1, 130, 128)), 148), ([1], 1),
+])
+def test_work_split_partition(tiles, C):
+    """Ranges partition [0, T) into near-equal pieces; every unit is touched by the
+    contiguous ranges [first, last]; at most one cut unit begins in any range, which
+    bounds the partial slots at two per range."""
+    starts, first, last = ops.work_split([int(t) for t in tiles], C)
+    T = int(sum(tiles))
+    assert starts[0] == 0 and starts[-1] == T
+    sizes = np.diff(starts)
+    assert sizes.min() >= T // C and sizes.max() <= -(-T // C)
+    Tu = np.concatenate([[0], np.cumsum(tiles)])
+    for u in range(len(tiles)):
+        # brute force: ranges whose [start, end) meets [Tu, Tu + tiles)
+        touching = [c for c in range(C) if starts[c] < Tu[u + 1] and starts[c + 1] > Tu[u]]
+        assert touching == list(range(first[u], last[u] + 1))
+    cut_starts = [first[u] for u in range(len(tiles)) if last[u] > first[u]]
+    assert len(cut_starts) == len(set(cut_starts))
+
+
+def test_no_device_plan_creation_reports_cuda_error():
+    """Without a visible GPU a valid descriptor yields TT_ERR_CUDA (never a CPU path)."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("GPU present")
+    import ctypes
+    desc = ops.Desc(1, 4, 1, 64, 16, 256, 0, 0.0, 0, 0, 0, 0)
+    h = ctypes.c_void_p()
+    st = ops.lib().tt_block_attn_plan(ctypes.byref(desc), 0, ctypes.byref(h))
+    assert st in (ops.TT_ERR_CUDA, ops.TT_ERR_INVALID_ARG)
+    assert not h.value

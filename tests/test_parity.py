@@ -1,0 +1,238 @@
+"""GPU parity: the CUDA kernels through the C ABI against the float64 oracle.
+
+Tolerance (bf16 inputs, fp32 accumulation): max-abs <= 1e-2 and relative
+L2 <= 5e-3, on `out` and on `lse`.  Context rows beyond L_n are NaN on the
+device in every decode case, so any read of them would show.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import block_attn as oracle_attn
+from oracle import block_causal as oracle_causal
+from tests.gpu_util import assert_parity, dev, f64, poison_beyond
+from two_tower_block_b200 import ops
+from two_tower_block_b200.workloads import WORKLOADS, make_causal, make_decode, make_workload
+
+pytestmark = pytest.mark.gpu
+
+KERNELS = [pytest.param(ops.KERNEL_TCGEN05, id="tcgen05"), pytest.param(ops.KERNEL_MMA_SYNC, id="mma_sync")]
+
+
+def run_decode(inp, kernel, num_ctas=0, poison=True):
+    B, S, Hq, Hkv, D, Lcap = inp.shape
+    plan = ops.Plan(B, Hq, Hkv, D, S, ctx_capacity=Lcap, kernel=kernel, num_ctas=num_ctas)
+    kc = poison_beyond(inp.k_ctx, inp.ctx_lens) if poison else inp.k_ctx
+    vc = poison_beyond(inp.v_ctx, inp.ctx_lens) if poison else inp.v_ctx
+    out, lse = plan.block_attn(dev(inp.q), dev(kc), dev(vc), dev(inp.k_blk), dev(inp.v_blk),
+                               torch.from_numpy(inp.ctx_lens).cuda(), want_lse=True)
+    plan.check()
+    return out, lse
+
+
+def oracle_decode(inp, idx=None):
+    sl = slice(None) if idx is None else idx
+    return oracle_attn(f64(inp.q[sl]), f64(inp.k_ctx[sl]), f64(inp.v_ctx[sl]), f64(inp.k_blk[sl]),
+                       f64(inp.v_blk[sl]), inp.ctx_lens[sl])
+
+
+SMALL = {
+    "tiny-workload": lambda: make_workload(1),
+    "gqa16-ragged": lambda: make_decode(3, 16, 32, 2, 128, 777, seed=7, ctx_lens=[0, 300, 777]),
+    "d64-g4": lambda: make_decode(2, 16, 8, 2, 64, 200, seed=8, ctx_lens=[129, 64]),
+    "odd-block-S5-g3": lambda: make_decode(2, 5, 6, 2, 128, 150, seed=9, ctx_lens=[150, 1]),
+    "S256-g1": lambda: make_decode(1, 256, 2, 2, 64, 300, seed=10, ctx_lens=[300]),
+    "S1-g16": lambda: make_decode(4, 1, 16, 1, 128, 513, seed=11, ctx_lens=[513, 0, 1, 255]),
+    "no-context": lambda: make_decode(2, 16, 4, 1, 64, 0, seed=12),
+    "peaky-std3": lambda: make_decode(2, 16, 16, 1, 128, 400, seed=13, std=3.0, peaky_frac=0.05,
+                                      ctx_lens=[400, 385]),
+}
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+@pytest.mark.parametrize("case", list(SMALL))
+def test_decode_small(case, kernel):
+    inp = SMALL[case]()
+    out, lse = run_decode(inp, kernel)
+    ro, rl = oracle_decode(inp)
+    assert_parity(out, ro, f"{case} out")
+    assert_parity(lse, rl, f"{case} lse")
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+@pytest.mark.parametrize("num_ctas", [1, 3, 37, 148, 300])
+def test_split_count_invariance(kernel, num_ctas):
+    """Any cut of the key list into segments recombines to the same softmax."""
+    inp = make_decode(3, 16, 32, 2, 128, 1000, seed=21, ctx_lens=[1000, 517, 3])
+    out, lse = run_decode(inp, kernel, num_ctas=num_ctas)
+    ro, rl = oracle_decode(inp)
+    assert_parity(out, ro, f"C={num_ctas} out")
+    assert_parity(lse, rl, f"C={num_ctas} lse")
+
+
+@pytest.fixture(scope="module")
+def wl2():
+    return make_workload(2)
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_decode_L4096_peaky_full(wl2, kernel):
+    """Full decode workload (B=8, Hq=32, Hkv=2, D=128, L=4096, 1% keys x8): every output."""
+    out, lse = run_decode(wl2, kernel)
+    ro, rl = oracle_decode(wl2)
+    assert_parity(out, ro, "L4096 out")
+    assert_parity(lse, rl, "L4096 lse")
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_decode_ragged_B64_sampled(kernel):
+    """Full ragged workload on the GPU; oracle on sampled sequences (shortest,
+    longest, first, one more)."""
+    inp = make_workload(3)
+    out, lse = run_decode(inp, kernel, poison=True)
+    lens = inp.ctx_lens
+    for n in sorted({int(np.argmin(lens)), int(np.argmax(lens)), 0, 33}):
+        ro, rl = oracle_decode(inp, slice(n, n + 1))
+        assert_parity(out[n:n + 1], ro, f"ragged n={n} L={lens[n]} out")
+        assert_parity(lse[n:n + 1], rl, f"ragged n={n} lse")
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_decode_long_L131072_sampled(kernel):
+    """Full long-context workload (B=4, L=131072, std 0.5) on the GPU; oracle on
+    sequence 2 (both KV heads), which spans many segments."""
+    inp = make_workload(4)
+    out, lse = run_decode(inp, kernel, poison=False)
+    assert torch.isfinite(out).all()
+    ro, rl = oracle_decode(inp, slice(2, 3))
+    assert_parity(out[2:3], ro, "long out")
+    assert_parity(lse[2:3], rl, "long lse")
+
+
+def run_causal(inp, kernel, num_ctas=0):
+    B, N, Hq, D = inp.q.shape
+    Hkv = inp.k_ctx.shape[1]
+    plan = ops.Plan(B, Hq, Hkv, D, inp.block_size, seq_len=N, kernel=kernel, num_ctas=num_ctas)
+    out, lse = plan.block_attn_block_causal(dev(inp.q), dev(inp.k_ctx), dev(inp.v_ctx), dev(inp.k_blk),
+                                            dev(inp.v_blk), want_lse=True)
+    plan.check()
+    return out, lse
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+@pytest.mark.parametrize("shape", [(2, 64, 16, 8, 2, 128), (1, 40, 4, 8, 1, 64), (2, 300, 20, 4, 2, 128)],
+                         ids=["S16-g4", "S4-g8-d64", "S20-g2"])
+def test_block_causal_small(kernel, shape):
+    B, N, S, Hq, Hkv, D = shape
+    inp = make_causal(B, N, S, Hq, Hkv, D, seed=31)
+    out, lse = run_causal(inp, kernel)
+    ro, rl = oracle_causal(f64(inp.q), f64(inp.k_ctx), f64(inp.v_ctx), f64(inp.k_blk), f64(inp.v_blk), S)
+    assert_parity(out, ro, "causal out")
+    assert_parity(lse, rl, "causal lse")
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_block_causal_full_sampled(kernel):
+    """Full training/prefill workload (B=8, N=8192, 512 blocks of 16) on the GPU;
+    oracle on sampled blocks of two sequences."""
+    w = WORKLOADS[5]
+    inp = make_workload(5)
+    out, lse = run_causal(inp, kernel)
+    S = w.block_size
+    for n, blocks in [(0, [0, 1, 8, 100, 511]), (7, [255, 511])]:
+        sl = slice(n, n + 1)
+        ro, rl = oracle_causal(f64(inp.q[sl]), f64(inp.k_ctx[sl]), f64(inp.v_ctx[sl]), f64(inp.k_blk[sl]),
+                               f64(inp.v_blk[sl]), S, blocks=blocks)
+        for b in blocks:
+            p = slice(S * b, S * b + S)
+            assert_parity(out[n:n + 1, p], ro[:, p], f"causal n={n} b={b} out")
+            assert_parity(lse[n:n + 1, :, p], rl[:, :, p], f"causal n={n} b={b} lse")
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_block_causal_equals_decode(kernel):
+    """Block b of the block-causal entry is the decode entry with L = S*b on the
+    same sequence (GPU against GPU, same kernel)."""
+    B, N, S, Hq, Hkv, D = 2, 96, 16, 8, 2, 128
+    inp = make_causal(B, N, S, Hq, Hkv, D, seed=41)
+    out_c, lse_c = run_causal(inp, kernel)
+    for b in [0, 1, 5]:
+        p = slice(S * b, S * b + S)
+        plan = ops.Plan(B, Hq, Hkv, D, S, ctx_capacity=N, kernel=kernel)
+        lens = torch.full((B,), S * b, dtype=torch.int32, device="cuda")
+        out_d, lse_d = plan.block_attn(dev(np.ascontiguousarray(inp.q[:, p])), dev(inp.k_ctx), dev(inp.v_ctx),
+                                       dev(np.ascontiguousarray(inp.k_blk[:, p])),
+                                       dev(np.ascontiguousarray(inp.v_blk[:, p])), lens, want_lse=True)
+        plan.check()
+        torch.testing.assert_close(out_d, out_c[:, p], atol=2e-5, rtol=1e-4)
+        torch.testing.assert_close(lse_d, lse_c[:, :, p], atol=2e-5, rtol=1e-4)
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_host_io_entry_matches_device_entry(kernel):
+    inp = make_decode(2, 16, 32, 2, 128, 600, seed=51, ctx_lens=[600, 257])
+    B, S, Hq, Hkv, D, Lcap = inp.shape
+    out_dev, lse_dev = run_decode(inp, kernel, poison=False)
+    plan = ops.Plan(B, Hq, Hkv, D, S, ctx_capacity=Lcap, kernel=kernel, host_io=True)
+
+    def pinned(bits):
+        return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+    out = torch.empty((B, S, Hq, D), dtype=torch.float32).pin_memory()
+    lse = torch.empty((B, Hq, S), dtype=torch.float32).pin_memory()
+    plan.block_attn_host(pinned(inp.q), pinned(inp.k_ctx), pinned(inp.v_ctx), pinned(inp.k_blk),
+                         pinned(inp.v_blk), torch.from_numpy(inp.ctx_lens).pin_memory(), out, lse)
+    plan.check()
+    torch.testing.assert_close(out, out_dev.cpu(), atol=0, rtol=0)
+    torch.testing.assert_close(lse, lse_dev.cpu(), atol=0, rtol=0)
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_ctx_len_out_of_range_is_reported(kernel):
+    inp = make_decode(2, 16, 8, 2, 64, 100, seed=61, ctx_lens=[100, 50])
+    B, S, Hq, Hkv, D, Lcap = inp.shape
+    plan = ops.Plan(B, Hq, Hkv, D, S, ctx_capacity=Lcap, kernel=kernel)
+    args = [dev(inp.q), dev(inp.k_ctx), dev(inp.v_ctx), dev(inp.k_blk), dev(inp.v_blk)]
+    bad = torch.tensor([101, 50], dtype=torch.int32, device="cuda")
+    plan.block_attn(*args, bad)
+    assert plan.check_status() == ops.TT_ERR_DEVICE_ARG
+    bad = torch.tensor([-3, 50], dtype=torch.int32, device="cuda")
+    plan.block_attn(*args, bad)
+    assert plan.check_status() == ops.TT_ERR_DEVICE_ARG
+    # the error word was cleared and the context still works
+    out = plan.block_attn(*args, torch.from_numpy(inp.ctx_lens).cuda())
+    plan.check()
+    ro, _ = oracle_decode(inp)
+    assert_parity(out, ro, "after device error")
+
+
+def test_wait_timeout_selftest():
+    """A wait on a barrier nothing arrives at gives up after its limit and reports
+    TT_ERR_TIMEOUT; the device stays usable."""
+    assert ops.selftest_wait_timeout(0, 20000) == ops.TT_ERR_TIMEOUT
+    x = torch.ones(1024, device="cuda")
+    assert float(x.sum()) == 1024.0
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_empty_batch_is_noop(kernel):
+    plan = ops.Plan(0, 8, 2, 128, 16, ctx_capacity=64, kernel=kernel)
+    e = torch.empty(0, dtype=torch.bfloat16, device="cuda")
+    lens = torch.empty(0, dtype=torch.int32, device="cuda")
+    out = torch.empty(0, dtype=torch.float32, device="cuda")
+    plan.block_attn(e, e, e, e, e, lens, out=out)
+    plan.check()
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_profile_hook_counts_launches(kernel):
+    inp = make_decode(2, 16, 32, 2, 128, 2048, seed=71)
+    B, S, Hq, Hkv, D, Lcap = inp.shape
+    plan = ops.Plan(B, Hq, Hkv, D, S, ctx_capacity=Lcap, kernel=kernel)
+    args = [dev(inp.q), dev(inp.k_ctx), dev(inp.v_ctx), dev(inp.k_blk), dev(inp.v_blk),
+            torch.from_numpy(inp.ctx_lens).cuda()]
+    plan.profile(True)
+    for _ in range(5):
+        plan.block_attn(*args)
+    n, ms = plan.profile_read(0)
+    plan.profile(False)
+    assert n == 5 and ms > 0

@@ -1,0 +1,540 @@
+// C ABI of the block attention library: plans, argument checks, launches,
+// host-buffer entry, device error word, per-kernel timing hook.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "../../include/tt_block_attn.h"
+#include "problem.h"
+#include "errbits.h"
+#include "sched.cuh"
+
+namespace {
+
+thread_local std::string g_detail;
+
+tt_status_t fail(tt_status_t st, const std::string& why) {
+  g_detail = why;
+  return st;
+}
+tt_status_t cuda_fail(cudaError_t e, const char* where) {
+  g_detail = std::string(where) + ": " + cudaGetErrorString(e);
+  return TT_ERR_CUDA;
+}
+
+// ---------------------------------------------------------- TMA encoding --
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// bf16 tensor map with `rank` dims (innermost first), 128-byte swizzle.
+bool encode_bf16(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, const uint64_t* strides_bytes,
+                 const uint32_t* box) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t d[5], s[4];
+  cuuint32_t b[5], e[5];
+  for (int i = 0; i < rank; ++i) {
+    d[i] = dims[i];
+    b[i] = box[i];
+    e[i] = 1;
+  }
+  for (int i = 0; i < rank - 1; ++i) s[i] = strides_bytes[i];
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base), d, s, b, e,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+constexpr int kProfMax = 4096;
+
+}  // namespace
+
+struct tt_plan_s {
+  tt_block_attn_desc desc;
+  int device = 0;
+  int sm_count = 0;
+  int kernel = TT_KERNEL_MMA_SYNC;
+  int C = 1;
+  int key_tile = 64;
+  int R = 0, g = 1;
+  float scale = 0.f;
+  // scratch
+  void* ws = nullptr;
+  size_t ws_bytes = 0;
+  float* part_o = nullptr;
+  float* part_lse = nullptr;
+  tt::SplitRecord* records = nullptr;
+  unsigned* err_word = nullptr;
+  int* causal_pref = nullptr;
+  long long causal_T = 0;
+  int causal_NB = 0;
+  // host IO staging
+  void* stage = nullptr;
+  size_t st_q = 0, st_kc = 0, st_kb = 0, st_lens = 0, st_out = 0, st_lse = 0;
+  // timing hook
+  bool prof_on = false;
+  std::vector<cudaEvent_t> prof_ev;      // 2 * kProfMax
+  std::vector<int> prof_kid;
+  int prof_n = 0;
+};
+
+namespace {
+
+struct DeviceGuard {
+  int prev = -1;
+  explicit DeviceGuard(int dev) {
+    if (cudaGetDevice(&prev) == cudaSuccess && prev != dev) cudaSetDevice(dev);
+    else prev = -1;
+  }
+  ~DeviceGuard() {
+    if (prev >= 0) cudaSetDevice(prev);
+  }
+};
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+void prof_mark(tt_plan_t plan, int kid, cudaStream_t s, bool begin) {
+  if (!plan->prof_on) return;
+  if (begin) {
+    if (plan->prof_n >= kProfMax) return;
+    cudaEventRecord(plan->prof_ev[2 * plan->prof_n], s);
+    plan->prof_kid[plan->prof_n] = kid;
+  } else {
+    if (plan->prof_n >= kProfMax) return;
+    cudaEventRecord(plan->prof_ev[2 * plan->prof_n + 1], s);
+    plan->prof_n++;
+  }
+}
+
+tt::Problem base_problem(tt_plan_t plan) {
+  tt::Problem p{};
+  const tt_block_attn_desc& d = plan->desc;
+  p.B = d.batch;
+  p.Hq = d.num_q_heads;
+  p.Hkv = d.num_kv_heads;
+  p.g = plan->g;
+  p.D = d.head_dim;
+  p.S = d.block_size;
+  p.R = plan->R;
+  p.scale_log2 = plan->scale * 1.4426950408889634f;
+  p.C = plan->C;
+  p.key_tile = plan->key_tile;
+  p.blk_tiles = tt::ceil_div(d.block_size, plan->key_tile);
+  p.part_o = plan->part_o;
+  p.part_lse = plan->part_lse;
+  p.records = plan->records;
+  p.err_word = plan->err_word;
+  p.wait_limit_ns = (unsigned long long)(d.wait_timeout_us > 0 ? d.wait_timeout_us : 1000000) * 1000ull;
+  return p;
+}
+
+tt_status_t launch_all(tt_plan_t plan, const tt::Problem& p, cudaStream_t s) {
+  cudaError_t e;
+  prof_mark(plan, 0, s, true);
+  if (plan->kernel == TT_KERNEL_TCGEN05) {
+    tt::TmaMaps maps;
+    memset(&maps, 0, sizeof(maps));
+    const uint64_t D = p.D;
+    const uint32_t g = p.g, S = p.S, kt = p.key_tile;
+    // q viewed as [tokens][Hq][D]; box = one unit's rows (S tokens x g heads x 64 dims)
+    {
+      uint64_t dims[3] = {D, (uint64_t)p.Hq, (uint64_t)p.B * p.NB * p.S};
+      uint64_t str[2] = {D * 2, (uint64_t)p.Hq * D * 2};
+      uint32_t box[3] = {64, g, S};
+      if (!encode_bf16(&maps.q, p.q, 3, dims, str, box)) return fail(TT_ERR_CUDA, "tensor map (q) encode failed");
+    }
+    // k_blk / v_blk viewed as [tokens][Hkv][D]; box = min(S, key_tile) tokens of one head
+    {
+      uint64_t dims[3] = {D, (uint64_t)p.Hkv, (uint64_t)p.B * p.NB * p.S};
+      uint64_t str[2] = {D * 2, (uint64_t)p.Hkv * D * 2};
+      uint32_t box[3] = {64, 1, std::min(S, kt)};
+      if (!encode_bf16(&maps.k_blk, p.k_blk, 3, dims, str, box) ||
+          !encode_bf16(&maps.v_blk, p.v_blk, 3, dims, str, box))
+        return fail(TT_ERR_CUDA, "tensor map (block kv) encode failed");
+    }
+    // k_ctx / v_ctx viewed as [B*Hkv*stride rows][D]; box = key_tile rows x 64 dims
+    if ((uint64_t)p.B * p.Hkv * p.ctx_stride > 0) {
+      uint64_t dims[2] = {D, (uint64_t)p.B * p.Hkv * p.ctx_stride};
+      uint64_t str[1] = {D * 2};
+      uint32_t box[2] = {64, kt};
+      if (!encode_bf16(&maps.k_ctx, p.k_ctx, 2, dims, str, box) ||
+          !encode_bf16(&maps.v_ctx, p.v_ctx, 2, dims, str, box))
+        return fail(TT_ERR_CUDA, "tensor map (context kv) encode failed");
+    } else {
+      maps.k_ctx = maps.k_blk;  // never read: no context tiles exist
+      maps.v_ctx = maps.v_blk;
+    }
+    e = tt::launch_attn_tcgen05(p, maps, s);
+  } else {
+    e = tt::launch_attn_mma_sync(p, s);
+  }
+  prof_mark(plan, 0, s, false);
+  if (e != cudaSuccess) return cuda_fail(e, "attention kernel launch");
+  if (plan->C > 1) {
+    prof_mark(plan, 1, s, true);
+    e = tt::launch_combine(p, s);
+    prof_mark(plan, 1, s, false);
+    if (e != cudaSuccess) return cuda_fail(e, "combine kernel launch");
+  }
+  return TT_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* tt_status_string(tt_status_t s) {
+  switch (s) {
+    case TT_OK: return "ok";
+    case TT_ERR_INVALID_ARG: return "invalid argument";
+    case TT_ERR_UNSUPPORTED: return "unsupported configuration";
+    case TT_ERR_CUDA: return "CUDA error";
+    case TT_ERR_DEVICE_ARG: return "device-side argument error (ctx_lens out of range)";
+    case TT_ERR_TIMEOUT: return "device-side pipeline wait timed out";
+  }
+  return "unknown status";
+}
+
+const char* tt_last_error_detail(void) { return g_detail.c_str(); }
+
+tt_status_t tt_block_attn_plan(const tt_block_attn_desc* desc, int device, tt_plan_t* out_plan) {
+  g_detail.clear();
+  if (!desc || !out_plan) return fail(TT_ERR_INVALID_ARG, "null descriptor or output pointer");
+  const tt_block_attn_desc d = *desc;
+  if (d.batch < 0 || d.num_q_heads < 1 || d.num_kv_heads < 1 || d.block_size < 1 || d.ctx_capacity < 0 ||
+      d.seq_len < 0 || d.num_ctas < 0 || d.wait_timeout_us < 0)
+    return fail(TT_ERR_INVALID_ARG, "negative or zero size in descriptor");
+  if (d.num_q_heads % d.num_kv_heads) return fail(TT_ERR_INVALID_ARG, "num_q_heads % num_kv_heads != 0");
+  if (!(d.scale >= 0.f) || std::isinf(d.scale)) return fail(TT_ERR_INVALID_ARG, "scale must be finite and >= 0");
+  if (d.seq_len % d.block_size) return fail(TT_ERR_INVALID_ARG, "seq_len % block_size != 0");
+  if (d.kernel < TT_KERNEL_AUTO || d.kernel > TT_KERNEL_MMA_SYNC) return fail(TT_ERR_INVALID_ARG, "unknown kernel");
+  if (d.flags & ~TT_PLAN_HOST_IO) return fail(TT_ERR_INVALID_ARG, "unknown flag bits");
+  if (d.head_dim != 64 && d.head_dim != 128) return fail(TT_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
+  const int g = d.num_q_heads / d.num_kv_heads;
+  if ((long long)d.block_size * g > 256) return fail(TT_ERR_UNSUPPORTED, "block_size * (Hq/Hkv) must be <= 256");
+  const long long tok = (long long)d.batch * std::max(d.seq_len, d.block_size);
+  if ((long long)d.batch * d.num_kv_heads * std::max(d.ctx_capacity, d.seq_len) > (1ll << 31) - 1 ||
+      tok * d.num_q_heads > (1ll << 31) - 1)
+    return fail(TT_ERR_UNSUPPORTED, "tensor too large (rows beyond 2^31)");
+
+  int ndev = 0;
+  cudaError_t e = cudaGetDeviceCount(&ndev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDeviceCount");
+  if (device < 0 || device >= ndev) return fail(TT_ERR_INVALID_ARG, "bad device ordinal");
+  DeviceGuard guard(device);
+  cudaDeviceProp prop;
+  e = cudaGetDeviceProperties(&prop, device);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDeviceProperties");
+
+  tt_plan_s* P = new tt_plan_s();
+  P->desc = d;
+  P->device = device;
+  P->sm_count = prop.multiProcessorCount;
+  P->g = g;
+  P->R = d.block_size * g;
+  P->scale = d.scale > 0.f ? d.scale : 1.0f / std::sqrt((float)d.head_dim);
+  P->kernel = d.kernel == TT_KERNEL_AUTO ? TT_KERNEL_MMA_SYNC : d.kernel;
+  if (P->kernel == TT_KERNEL_TCGEN05 && prop.major != 10) P->kernel = TT_KERNEL_MMA_SYNC;
+  if (P->kernel == TT_KERNEL_TCGEN05) {
+    P->key_tile = 128;
+    P->C = d.num_ctas > 0 ? d.num_ctas : P->sm_count;
+  } else {
+    P->key_tile = 64;
+    const int rb = (P->R + 63) / 64;
+    P->C = d.num_ctas > 0 ? d.num_ctas : std::max(1, (4 * P->sm_count) / rb);
+  }
+
+  // block-causal tile prefix over block index b (identical for every (n, h))
+  std::vector<int> pref;
+  if (d.seq_len > 0) {
+    const int NB = d.seq_len / d.block_size;
+    pref.resize(NB + 1);
+    long long acc = 0;
+    for (int b = 0; b <= NB; ++b) {
+      pref[b] = (int)acc;
+      if (b < NB) acc += tt::ceil_div(d.block_size, P->key_tile) + tt::ceil_div(d.block_size * b, P->key_tile);
+    }
+    if (acc > (1ll << 31) - 1) {
+      delete P;
+      return fail(TT_ERR_UNSUPPORTED, "sequence too long");
+    }
+    P->causal_NB = NB;
+    P->causal_T = (long long)d.batch * d.num_kv_heads * acc;
+  }
+
+  // scratch layout (256-byte aligned pieces)
+  auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  const size_t b_po = up((size_t)2 * P->C * P->R * d.head_dim * sizeof(float));
+  const size_t b_pl = up((size_t)2 * P->C * P->R * sizeof(float));
+  const size_t b_rec = up((size_t)P->C * sizeof(tt::SplitRecord));
+  const size_t b_err = 256;
+  const size_t b_pref = up(pref.size() * sizeof(int));
+  P->ws_bytes = b_po + b_pl + b_rec + b_err + b_pref;
+  e = cudaMalloc(&P->ws, P->ws_bytes);
+  if (e != cudaSuccess) {
+    delete P;
+    return cuda_fail(e, "cudaMalloc(workspace)");
+  }
+  char* w = static_cast<char*>(P->ws);
+  P->part_o = reinterpret_cast<float*>(w);
+  P->part_lse = reinterpret_cast<float*>(w + b_po);
+  P->records = reinterpret_cast<tt::SplitRecord*>(w + b_po + b_pl);
+  P->err_word = reinterpret_cast<unsigned*>(w + b_po + b_pl + b_rec);
+  P->causal_pref = pref.empty() ? nullptr : reinterpret_cast<int*>(w + b_po + b_pl + b_rec + b_err);
+  e = cudaMemset(P->err_word, 0, b_err);
+  if (e == cudaSuccess && !pref.empty())
+    e = cudaMemcpy(P->causal_pref, pref.data(), pref.size() * sizeof(int), cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) {
+    cudaFree(P->ws);
+    delete P;
+    return cuda_fail(e, "workspace init");
+  }
+
+  if (d.flags & TT_PLAN_HOST_IO) {
+    const size_t B = d.batch, S = d.block_size, Hq = d.num_q_heads, Hkv = d.num_kv_heads, D = d.head_dim;
+    P->st_q = up(B * S * Hq * D * 2);
+    P->st_kc = up(B * Hkv * (size_t)d.ctx_capacity * D * 2);
+    P->st_kb = up(B * S * Hkv * D * 2);
+    P->st_lens = up(B * 4);
+    P->st_out = up(B * S * Hq * D * 4);
+    P->st_lse = up(B * Hq * S * 4);
+    const size_t tot = P->st_q + 2 * P->st_kc + 2 * P->st_kb + P->st_lens + P->st_out + P->st_lse;
+    e = cudaMalloc(&P->stage, std::max<size_t>(tot, 256));
+    if (e != cudaSuccess) {
+      cudaFree(P->ws);
+      delete P;
+      return cuda_fail(e, "cudaMalloc(host-io staging)");
+    }
+  }
+  *out_plan = P;
+  return TT_OK;
+}
+
+void tt_block_attn_plan_destroy(tt_plan_t plan) {
+  if (!plan) return;
+  DeviceGuard guard(plan->device);
+  for (cudaEvent_t ev : plan->prof_ev) cudaEventDestroy(ev);
+  if (plan->ws) cudaFree(plan->ws);
+  if (plan->stage) cudaFree(plan->stage);
+  delete plan;
+}
+
+tt_status_t tt_block_attn_plan_get_info(tt_plan_t plan, tt_plan_info* info) {
+  if (!plan || !info) return fail(TT_ERR_INVALID_ARG, "null plan or info");
+  info->kernel = plan->kernel;
+  info->num_ctas = plan->C;
+  info->key_tile = plan->key_tile;
+  info->rows_per_unit = plan->R;
+  info->workspace_bytes = plan->ws_bytes;
+  info->sm_count = plan->sm_count;
+  return TT_OK;
+}
+
+tt_status_t tt_block_attn(tt_plan_t plan, const void* q, const void* k_ctx, const void* v_ctx, const void* k_blk,
+                          const void* v_blk, const int32_t* ctx_lens, float* out, float* lse, tt_stream_t stream) {
+  if (!plan) return fail(TT_ERR_INVALID_ARG, "null plan");
+  const tt_block_attn_desc& d = plan->desc;
+  if (d.batch == 0) return TT_OK;
+  if (!q || !k_blk || !v_blk || !ctx_lens || !out) return fail(TT_ERR_INVALID_ARG, "null tensor pointer");
+  if (d.ctx_capacity > 0 && (!k_ctx || !v_ctx)) return fail(TT_ERR_INVALID_ARG, "null context pointer");
+  if (!aligned16(q) || !aligned16(k_ctx) || !aligned16(v_ctx) || !aligned16(k_blk) || !aligned16(v_blk) ||
+      !aligned16(out) || !aligned16(lse) || (reinterpret_cast<uintptr_t>(ctx_lens) & 3u))
+    return fail(TT_ERR_INVALID_ARG, "tensor pointer not 16-byte aligned");
+  DeviceGuard guard(plan->device);
+  tt::Problem p = base_problem(plan);
+  p.mode = tt::kDecode;
+  p.NB = 1;
+  p.ctx_stride = d.ctx_capacity;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.k_ctx = static_cast<const __nv_bfloat16*>(k_ctx);
+  p.v_ctx = static_cast<const __nv_bfloat16*>(v_ctx);
+  p.k_blk = static_cast<const __nv_bfloat16*>(k_blk);
+  p.v_blk = static_cast<const __nv_bfloat16*>(v_blk);
+  p.ctx_lens = ctx_lens;
+  p.out = out;
+  p.lse = lse;
+  return launch_all(plan, p, reinterpret_cast<cudaStream_t>(stream));
+}
+
+tt_status_t tt_block_attn_block_causal(tt_plan_t plan, const void* q, const void* k_ctx, const void* v_ctx,
+                                       const void* k_blk, const void* v_blk, float* out, float* lse,
+                                       tt_stream_t stream) {
+  if (!plan) return fail(TT_ERR_INVALID_ARG, "null plan");
+  const tt_block_attn_desc& d = plan->desc;
+  if (d.seq_len == 0) return fail(TT_ERR_INVALID_ARG, "plan has seq_len == 0 (decode-only)");
+  if (d.batch == 0) return TT_OK;
+  if (!q || !k_ctx || !v_ctx || !k_blk || !v_blk || !out) return fail(TT_ERR_INVALID_ARG, "null tensor pointer");
+  if (!aligned16(q) || !aligned16(k_ctx) || !aligned16(v_ctx) || !aligned16(k_blk) || !aligned16(v_blk) ||
+      !aligned16(out) || !aligned16(lse))
+    return fail(TT_ERR_INVALID_ARG, "tensor pointer not 16-byte aligned");
+  DeviceGuard guard(plan->device);
+  tt::Problem p = base_problem(plan);
+  p.mode = tt::kBlockCausal;
+  p.NB = plan->causal_NB;
+  p.ctx_stride = d.seq_len;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.k_ctx = static_cast<const __nv_bfloat16*>(k_ctx);
+  p.v_ctx = static_cast<const __nv_bfloat16*>(v_ctx);
+  p.k_blk = static_cast<const __nv_bfloat16*>(k_blk);
+  p.v_blk = static_cast<const __nv_bfloat16*>(v_blk);
+  p.ctx_lens = nullptr;
+  p.out = out;
+  p.lse = lse;
+  p.T_causal = plan->causal_T;
+  p.causal_pref = plan->causal_pref;
+  return launch_all(plan, p, reinterpret_cast<cudaStream_t>(stream));
+}
+
+tt_status_t tt_block_attn_host(tt_plan_t plan, const void* q, const void* k_ctx, const void* v_ctx, const void* k_blk,
+                               const void* v_blk, const int32_t* ctx_lens, float* out, float* lse,
+                               tt_stream_t stream) {
+  if (!plan) return fail(TT_ERR_INVALID_ARG, "null plan");
+  if (!plan->stage) return fail(TT_ERR_INVALID_ARG, "plan was created without TT_PLAN_HOST_IO");
+  const tt_block_attn_desc& d = plan->desc;
+  if (d.batch == 0) return TT_OK;
+  if (!q || !k_blk || !v_blk || !ctx_lens || !out || (d.ctx_capacity > 0 && (!k_ctx || !v_ctx)))
+    return fail(TT_ERR_INVALID_ARG, "null host pointer");
+  DeviceGuard guard(plan->device);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  char* st = static_cast<char*>(plan->stage);
+  const size_t B = d.batch, S = d.block_size, Hq = d.num_q_heads, Hkv = d.num_kv_heads, D = d.head_dim;
+  char* dq = st;
+  char* dkc = dq + plan->st_q;
+  char* dvc = dkc + plan->st_kc;
+  char* dkb = dvc + plan->st_kc;
+  char* dvb = dkb + plan->st_kb;
+  char* dl = dvb + plan->st_kb;
+  char* dout = dl + plan->st_lens;
+  char* dlse = dout + plan->st_out;
+  const size_t nq = B * S * Hq * D * 2, nkc = B * Hkv * (size_t)d.ctx_capacity * D * 2, nkb = B * S * Hkv * D * 2;
+  cudaError_t e = cudaSuccess;
+  // one cudaMemcpyAsync per buffer
+  if (e == cudaSuccess) e = cudaMemcpyAsync(dq, q, nq, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess && nkc) e = cudaMemcpyAsync(dkc, k_ctx, nkc, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess && nkc) e = cudaMemcpyAsync(dvc, v_ctx, nkc, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(dkb, k_blk, nkb, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(dvb, v_blk, nkb, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(dl, ctx_lens, B * 4, cudaMemcpyHostToDevice, s);
+  if (e != cudaSuccess) return cuda_fail(e, "host-to-device copy");
+  tt_status_t r = tt_block_attn(plan, dq, nkc ? dkc : nullptr, nkc ? dvc : nullptr, dkb, dvb,
+                                reinterpret_cast<const int32_t*>(dl), reinterpret_cast<float*>(dout),
+                                lse ? reinterpret_cast<float*>(dlse) : nullptr, stream);
+  if (r != TT_OK) return r;
+  e = cudaMemcpyAsync(out, dout, B * S * Hq * D * 4, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess && lse) e = cudaMemcpyAsync(lse, dlse, B * Hq * S * 4, cudaMemcpyDeviceToHost, s);
+  if (e != cudaSuccess) return cuda_fail(e, "device-to-host copy");
+  return TT_OK;
+}
+
+tt_status_t tt_block_attn_check(tt_plan_t plan, tt_stream_t stream) {
+  if (!plan) return fail(TT_ERR_INVALID_ARG, "null plan");
+  DeviceGuard guard(plan->device);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  unsigned w = 0;
+  e = cudaMemcpy(&w, plan->err_word, sizeof(w), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess) e = cudaMemset(plan->err_word, 0, sizeof(unsigned));
+  if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
+  if (w & tt::kErrTimeout) return fail(TT_ERR_TIMEOUT, "an in-kernel wait timed out");
+  if (w & tt::kErrDeviceArg) return fail(TT_ERR_DEVICE_ARG, "ctx_lens value outside [0, ctx_capacity]");
+  return TT_OK;
+}
+
+tt_status_t tt_block_attn_profile(tt_plan_t plan, int enable) {
+  if (!plan) return fail(TT_ERR_INVALID_ARG, "null plan");
+  DeviceGuard guard(plan->device);
+  if (enable && plan->prof_ev.empty()) {
+    plan->prof_ev.resize(2 * kProfMax);
+    plan->prof_kid.resize(kProfMax);
+    for (auto& ev : plan->prof_ev) {
+      cudaError_t e = cudaEventCreate(&ev);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaEventCreate");
+    }
+  }
+  plan->prof_on = enable != 0;
+  plan->prof_n = 0;
+  return TT_OK;
+}
+
+tt_status_t tt_block_attn_profile_read(tt_plan_t plan, int kernel_id, int* launches, double* total_ms) {
+  if (!plan || !launches || !total_ms) return fail(TT_ERR_INVALID_ARG, "null argument");
+  DeviceGuard guard(plan->device);
+  int n = 0;
+  double tot = 0.0;
+  for (int i = 0; i < plan->prof_n; ++i) {
+    if (plan->prof_kid[i] != kernel_id) continue;
+    cudaError_t e = cudaEventSynchronize(plan->prof_ev[2 * i + 1]);
+    float ms = 0.f;
+    if (e == cudaSuccess) e = cudaEventElapsedTime(&ms, plan->prof_ev[2 * i], plan->prof_ev[2 * i + 1]);
+    if (e != cudaSuccess) return cuda_fail(e, "reading profile events");
+    tot += ms;
+    ++n;
+  }
+  *launches = n;
+  *total_ms = tot;
+  plan->prof_n = 0;
+  return TT_OK;
+}
+
+tt_status_t tt_selftest_wait_timeout(int device, int timeout_us, tt_stream_t stream) {
+  if (timeout_us <= 0) return fail(TT_ERR_INVALID_ARG, "timeout_us must be > 0");
+  DeviceGuard guard(device);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  unsigned* w = nullptr;
+  cudaError_t e = cudaMalloc(&w, sizeof(unsigned));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc");
+  e = cudaMemsetAsync(w, 0, sizeof(unsigned), s);
+  if (e == cudaSuccess) e = tt::launch_wait_selftest(w, (unsigned long long)timeout_us * 1000ull, s);
+  unsigned h = 0;
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e == cudaSuccess) e = cudaMemcpy(&h, w, sizeof(h), cudaMemcpyDeviceToHost);
+  cudaFree(w);
+  if (e != cudaSuccess) return cuda_fail(e, "wait self test");
+  if (h & 0x80000000u) return fail(TT_ERR_INVALID_ARG, "self test: a wait on a barrier nothing arrives at returned");
+  if (h & tt::kErrTimeout) return TT_ERR_TIMEOUT;
+  return TT_OK;
+}
+
+tt_status_t tt_debug_work_split(int num_units, const int* tiles_per_unit, int num_ctas, long long* range_start,
+                                int* unit_first, int* unit_last) {
+  if (num_units < 0 || num_ctas < 1 || (num_units > 0 && (!tiles_per_unit || !unit_first || !unit_last)) ||
+      !range_start)
+    return fail(TT_ERR_INVALID_ARG, "bad arguments");
+  long long T = 0;
+  for (int u = 0; u < num_units; ++u) {
+    if (tiles_per_unit[u] < 1) return fail(TT_ERR_INVALID_ARG, "every unit has at least one tile");
+    T += tiles_per_unit[u];
+  }
+  for (int c = 0; c <= num_ctas; ++c) range_start[c] = tt::range_start(T, num_ctas, c);
+  long long Tu = 0;
+  for (int u = 0; u < num_units; ++u) {
+    unit_first[u] = tt::range_of_tile(T, num_ctas, Tu);
+    unit_last[u] = tt::range_of_tile(T, num_ctas, Tu + tiles_per_unit[u] - 1);
+    Tu += tiles_per_unit[u];
+  }
+  return TT_OK;
+}
+
+}  // extern "C"

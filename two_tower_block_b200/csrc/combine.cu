@@ -1,0 +1,98 @@
+// Log-sum-exp combine of the units that a range boundary cut into segments,
+// and the bounded-wait self test.
+//
+// A cut unit's segments each hold O_s = (sum over its keys of e^{s-m_s} v) /
+// l_s and lse_s = m_s + ln l_s.  The joint softmax over all keys of the unit
+// is recovered exactly: with M = max_s lse_s and w_s = e^{lse_s - M},
+//     out = sum_s w_s O_s / sum_s w_s,     lse = M + ln sum_s w_s.
+#include "problem.h"
+#include "ptx.cuh"
+#include "walker.cuh"
+
+namespace tt {
+namespace {
+
+constexpr int kRowsPerBlock = 16;
+constexpr int kThreads = 256;
+
+template <int D>
+__global__ void __launch_bounds__(kThreads) combine_kernel(const Problem p) {
+  const int c = blockIdx.x;
+  const SplitRecord rec = p.records[c];
+  if (rec.unit < 0) return;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const Unit x = make_unit(p, rec.unit, 0);
+  const int nseg = rec.last_range - c + 1;
+  constexpr int V = D / 32;  // columns per lane
+  const int r_end = min(p.R, (int)(blockIdx.y + 1) * kRowsPerBlock);
+  for (int r = blockIdx.y * kRowsPerBlock + warp; r < r_end; r += kThreads / 32) {
+    float M = -INFINITY;
+    for (int s = lane; s < nseg; s += 32) {
+      const int slot = s == 0 ? 2 * c + rec.first_which : 2 * (c + s);
+      M = fmaxf(M, p.part_lse[(size_t)slot * p.R + r]);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float acc[V];
+#pragma unroll
+    for (int v = 0; v < V; ++v) acc[v] = 0.f;
+    float wsum = 0.f;
+    for (int s = 0; s < nseg; ++s) {
+      const int slot = s == 0 ? 2 * c + rec.first_which : 2 * (c + s);
+      const float w = expf(p.part_lse[(size_t)slot * p.R + r] - M);
+      wsum += w;
+      const float* src = p.part_o + ((size_t)slot * p.R + r) * D + lane * V;
+      if constexpr (V == 4) {
+        const float4 a = *reinterpret_cast<const float4*>(src);
+        acc[0] += w * a.x; acc[1] += w * a.y; acc[2] += w * a.z; acc[3] += w * a.w;
+      } else {
+        const float2 a = *reinterpret_cast<const float2*>(src);
+        acc[0] += w * a.x; acc[1] += w * a.y;
+      }
+    }
+    const float inv = 1.f / wsum;
+    const int t = r / p.g, j = r - (r / p.g) * p.g;
+    float* dst = p.out + ((size_t)(x.ns * p.S + t) * p.Hq + x.h * p.g + j) * D + lane * V;
+    if constexpr (V == 4) {
+      *reinterpret_cast<float4*>(dst) = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+    } else {
+      *reinterpret_cast<float2*>(dst) = make_float2(acc[0] * inv, acc[1] * inv);
+    }
+    if (lane == 0 && p.lse)
+      p.lse[(size_t)(x.n * p.Hq + x.h * p.g + j) * (p.NB * p.S) + x.b * p.S + t] = M + logf(wsum);
+  }
+}
+
+// One thread waits on a barrier that nothing arrives at; the bounded wait must
+// give up, raise kErrTimeout and return.
+__global__ void wait_selftest_kernel(unsigned* err_word, unsigned long long limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    WaitCtx w{&abort_flag, err_word, limit_ns};
+    if (mbar_wait(smem_u32(&bar), 0, w)) atomicOr(err_word, 0x80000000u);  // must not happen
+  }
+  __syncthreads();
+}
+
+}  // namespace
+
+cudaError_t launch_combine(const Problem& p, cudaStream_t stream) {
+  dim3 grid(p.C, (p.R + kRowsPerBlock - 1) / kRowsPerBlock);
+  if (p.D == 128) combine_kernel<128><<<grid, kThreads, 0, stream>>>(p);
+  else combine_kernel<64><<<grid, kThreads, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_wait_selftest(unsigned* err_word, unsigned long long limit_ns, cudaStream_t stream) {
+  wait_selftest_kernel<<<1, 32, 0, stream>>>(err_word, limit_ns);
+  return cudaGetLastError();
+}
+
+}  // namespace tt

@@ -1,0 +1,56 @@
+// Problem description handed to every kernel (by value, as a kernel parameter).
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "sched.cuh"
+
+namespace tt {
+
+enum Mode : int { kDecode = 0, kBlockCausal = 1 };
+
+struct Problem {
+  // geometry
+  int mode;        // kDecode or kBlockCausal
+  int B, Hq, Hkv, g, D, S, R;  // R = S * g packed rows of one unit (row = t * g + j)
+  int NB;          // blocks per sequence: 1 for decode, N / S for block-causal
+  int ctx_stride;  // tokens per (n, h) slab of k_ctx / v_ctx: Lcap or N
+  float scale_log2;  // softmax scale * log2(e)
+  // tensors (caller-owned device memory)
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* k_ctx;
+  const __nv_bfloat16* v_ctx;
+  const __nv_bfloat16* k_blk;
+  const __nv_bfloat16* v_blk;
+  const int* ctx_lens;  // decode only
+  float* out;
+  float* lse;           // may be null
+  // work split
+  int C;                // ranges
+  int key_tile;         // keys per tile
+  int blk_tiles;        // tiles holding the block's own keys: ceil(S / key_tile)
+  long long T_causal;   // block-causal: total tiles (decode computes T on the device)
+  const int* causal_pref;  // block-causal: tiles before block b within one (n, h); NB + 1 entries
+  // plan-owned scratch
+  float* part_o;        // [2C][R][D]
+  float* part_lse;      // [2C][R]
+  SplitRecord* records; // [C]
+  unsigned* err_word;
+  unsigned long long wait_limit_ns;
+};
+
+// Host launchers (each returns the cudaError_t of its launch).
+cudaError_t launch_attn_mma_sync(const Problem& p, cudaStream_t stream);
+cudaError_t launch_combine(const Problem& p, cudaStream_t stream);
+cudaError_t launch_wait_selftest(unsigned* err_word, unsigned long long limit_ns, cudaStream_t stream);
+
+struct TmaMaps {
+  CUtensorMap q, k_ctx, v_ctx, k_blk, v_blk;
+};
+cudaError_t launch_attn_tcgen05(const Problem& p, const TmaMaps& maps, cudaStream_t stream);
+size_t attn_tcgen05_smem_bytes(int D);
+size_t attn_mma_sync_smem_bytes(int D);
+
+}  // namespace tt

@@ -1,0 +1,256 @@
+"""ctypes binding of libtt_block_attn.so (argument marshalling only).
+
+Every entry point here forwards to the C function of the same name in
+``include/tt_block_attn.h``.  torch supplies device memory and streams; all
+computation happens in the library's CUDA kernels.  If the library is
+missing, or a call is made without a CUDA device, the call raises: there is
+no CPU fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+__all__ = ["TTError", "Plan", "lib", "library_path", "block_attn", "block_attn_block_causal",
+           "selftest_wait_timeout", "work_split", "KERNEL_AUTO", "KERNEL_TCGEN05", "KERNEL_MMA_SYNC",
+           "TT_OK", "TT_ERR_INVALID_ARG", "TT_ERR_UNSUPPORTED", "TT_ERR_CUDA", "TT_ERR_DEVICE_ARG",
+           "TT_ERR_TIMEOUT", "EXPORTED_SYMBOLS"]
+
+TT_OK, TT_ERR_INVALID_ARG, TT_ERR_UNSUPPORTED, TT_ERR_CUDA, TT_ERR_DEVICE_ARG, TT_ERR_TIMEOUT = range(6)
+KERNEL_AUTO, KERNEL_TCGEN05, KERNEL_MMA_SYNC = 0, 1, 2
+PLAN_HOST_IO = 1
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+library_path = os.path.join(_HERE, "libtt_block_attn.so")
+
+# Every symbol the header declares (checked by the CPU test suite).
+EXPORTED_SYMBOLS = [
+    "tt_block_attn_plan", "tt_block_attn_plan_destroy", "tt_block_attn_plan_get_info", "tt_block_attn",
+    "tt_block_attn_block_causal", "tt_block_attn_host", "tt_block_attn_check", "tt_block_attn_profile",
+    "tt_block_attn_profile_read", "tt_selftest_wait_timeout", "tt_debug_work_split", "tt_status_string",
+    "tt_last_error_detail",
+]
+
+
+class Desc(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int), ("num_q_heads", ctypes.c_int), ("num_kv_heads", ctypes.c_int),
+                ("head_dim", ctypes.c_int), ("block_size", ctypes.c_int), ("ctx_capacity", ctypes.c_int),
+                ("seq_len", ctypes.c_int), ("scale", ctypes.c_float), ("kernel", ctypes.c_int),
+                ("num_ctas", ctypes.c_int), ("flags", ctypes.c_int), ("wait_timeout_us", ctypes.c_int)]
+
+
+class PlanInfo(ctypes.Structure):
+    _fields_ = [("kernel", ctypes.c_int), ("num_ctas", ctypes.c_int), ("key_tile", ctypes.c_int),
+                ("rows_per_unit", ctypes.c_int), ("workspace_bytes", ctypes.c_size_t),
+                ("sm_count", ctypes.c_int)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load the library once; raise (never fall back) if it is absent."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(library_path):
+        raise RuntimeError(f"{library_path} is missing: build it with `python -m two_tower_block_b200.build`")
+    L = ctypes.CDLL(library_path)
+    vp, ip, i, f = ctypes.c_void_p, ctypes.POINTER(ctypes.c_int), ctypes.c_int, ctypes.c_float
+    L.tt_block_attn_plan.argtypes = [ctypes.POINTER(Desc), i, ctypes.POINTER(vp)]
+    L.tt_block_attn_plan_destroy.argtypes = [vp]
+    L.tt_block_attn_plan_destroy.restype = None
+    L.tt_block_attn_plan_get_info.argtypes = [vp, ctypes.POINTER(PlanInfo)]
+    L.tt_block_attn.argtypes = [vp] * 10
+    L.tt_block_attn_block_causal.argtypes = [vp] * 9
+    L.tt_block_attn_host.argtypes = [vp] * 10
+    L.tt_block_attn_check.argtypes = [vp, vp]
+    L.tt_block_attn_profile.argtypes = [vp, i]
+    L.tt_block_attn_profile_read.argtypes = [vp, i, ip, ctypes.POINTER(ctypes.c_double)]
+    L.tt_selftest_wait_timeout.argtypes = [i, i, vp]
+    L.tt_debug_work_split.argtypes = [i, ip, i, ctypes.POINTER(ctypes.c_longlong), ip, ip]
+    L.tt_status_string.argtypes = [i]
+    L.tt_status_string.restype = ctypes.c_char_p
+    L.tt_last_error_detail.argtypes = []
+    L.tt_last_error_detail.restype = ctypes.c_char_p
+    for name in EXPORTED_SYMBOLS:
+        if name not in ("tt_block_attn_plan_destroy", "tt_status_string", "tt_last_error_detail"):
+            getattr(L, name).restype = ctypes.c_int
+    _lib = L
+    return L
+
+
+class TTError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        L = lib()
+        self.status = status
+        msg = L.tt_status_string(status).decode()
+        detail = L.tt_last_error_detail().decode()
+        super().__init__(f"{where}: {msg}" + (f" ({detail})" if detail else ""))
+
+
+def _check(status: int, where: str):
+    if status != TT_OK:
+        raise TTError(status, where)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, torch.Tensor):
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+        return ctypes.c_void_p(t.data_ptr())
+    return ctypes.c_void_p(int(t))
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+@dataclass
+class Shape:
+    batch: int
+    q_heads: int
+    kv_heads: int
+    head_dim: int
+    block: int
+    ctx_capacity: int = 0
+    seq_len: int = 0
+
+
+class Plan:
+    """Owns a tt_plan_t (device scratch, work split) for one shape on one device."""
+
+    def __init__(self, batch, q_heads, kv_heads, head_dim, block, ctx_capacity=0, seq_len=0, scale=0.0,
+                 kernel=KERNEL_AUTO, num_ctas=0, host_io=False, wait_timeout_us=0, device=None):
+        if device is None:
+            device = torch.cuda.current_device()
+        self.shape = Shape(batch, q_heads, kv_heads, head_dim, block, ctx_capacity, seq_len)
+        self.device = int(device)
+        d = Desc(batch, q_heads, kv_heads, head_dim, block, ctx_capacity, seq_len, float(scale), kernel,
+                 num_ctas, PLAN_HOST_IO if host_io else 0, wait_timeout_us)
+        h = ctypes.c_void_p()
+        _check(lib().tt_block_attn_plan(ctypes.byref(d), self.device, ctypes.byref(h)), "tt_block_attn_plan")
+        self._h = h
+
+    def close(self):
+        if getattr(self, "_h", None):
+            lib().tt_block_attn_plan_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def info(self) -> PlanInfo:
+        inf = PlanInfo()
+        _check(lib().tt_block_attn_plan_get_info(self._h, ctypes.byref(inf)), "tt_block_attn_plan_get_info")
+        return inf
+
+    # --- decode ------------------------------------------------------------
+    def block_attn(self, q, k_ctx, v_ctx, k_blk, v_blk, ctx_lens, out=None, lse=None, stream=None,
+                   want_lse=False):
+        s = self.shape
+        if out is None:
+            out = torch.empty((s.batch, s.block, s.q_heads, s.head_dim), dtype=torch.float32, device=q.device)
+        if lse is None and want_lse:
+            lse = torch.empty((s.batch, s.q_heads, s.block), dtype=torch.float32, device=q.device)
+        _check(lib().tt_block_attn(self._h, _ptr(q), _ptr(k_ctx), _ptr(v_ctx), _ptr(k_blk), _ptr(v_blk),
+                                   _ptr(ctx_lens), _ptr(out), _ptr(lse), _stream(stream)), "tt_block_attn")
+        return (out, lse) if want_lse or lse is not None else out
+
+    def block_attn_host(self, q, k_ctx, v_ctx, k_blk, v_blk, ctx_lens, out, lse=None, stream=None):
+        """Host (ideally pinned) CPU tensors in and out; copies happen inside the library."""
+        _check(lib().tt_block_attn_host(self._h, _ptr(q), _ptr(k_ctx), _ptr(v_ctx), _ptr(k_blk), _ptr(v_blk),
+                                        _ptr(ctx_lens), _ptr(out), _ptr(lse), _stream(stream)),
+               "tt_block_attn_host")
+        return out
+
+    # --- block-causal ------------------------------------------------------
+    def block_attn_block_causal(self, q, k_ctx, v_ctx, k_blk, v_blk, out=None, lse=None, stream=None,
+                                want_lse=False):
+        s = self.shape
+        if out is None:
+            out = torch.empty((s.batch, s.seq_len, s.q_heads, s.head_dim), dtype=torch.float32, device=q.device)
+        if lse is None and want_lse:
+            lse = torch.empty((s.batch, s.q_heads, s.seq_len), dtype=torch.float32, device=q.device)
+        _check(lib().tt_block_attn_block_causal(self._h, _ptr(q), _ptr(k_ctx), _ptr(v_ctx), _ptr(k_blk),
+                                                _ptr(v_blk), _ptr(out), _ptr(lse), _stream(stream)),
+               "tt_block_attn_block_causal")
+        return (out, lse) if want_lse or lse is not None else out
+
+    # --- status / timing ---------------------------------------------------
+    def check(self, stream=None):
+        """Synchronise and read the device error word; raise TTError on a device-side error."""
+        _check(lib().tt_block_attn_check(self._h, _stream(stream)), "tt_block_attn_check")
+
+    def check_status(self, stream=None) -> int:
+        return lib().tt_block_attn_check(self._h, _stream(stream))
+
+    def profile(self, enable: bool):
+        _check(lib().tt_block_attn_profile(self._h, int(enable)), "tt_block_attn_profile")
+
+    def profile_read(self, kernel_id: int):
+        n = ctypes.c_int()
+        ms = ctypes.c_double()
+        _check(lib().tt_block_attn_profile_read(self._h, kernel_id, ctypes.byref(n), ctypes.byref(ms)),
+               "tt_block_attn_profile_read")
+        return n.value, ms.value
+
+
+_plans = {}
+
+
+def _cached_plan(key, **kw):
+    p = _plans.get(key)
+    if p is None:
+        p = Plan(**kw)
+        _plans[key] = p
+    return p
+
+
+def block_attn(q, k_ctx, v_ctx, k_blk, v_blk, ctx_lens, scale=0.0, kernel=KERNEL_AUTO, want_lse=False):
+    """Decode block attention on torch CUDA tensors (shapes as in the C header)."""
+    B, S, Hq, D = q.shape
+    Hkv, Lcap = k_ctx.shape[1], k_ctx.shape[2]
+    dev = q.device.index if q.device.index is not None else torch.cuda.current_device()
+    key = ("dec", B, S, Hq, Hkv, D, Lcap, float(scale), kernel, dev)
+    plan = _cached_plan(key, batch=B, q_heads=Hq, kv_heads=Hkv, head_dim=D, block=S, ctx_capacity=Lcap,
+                        scale=scale, kernel=kernel, device=dev)
+    return plan.block_attn(q, k_ctx, v_ctx, k_blk, v_blk, ctx_lens, want_lse=want_lse)
+
+
+def block_attn_block_causal(q, k_ctx, v_ctx, k_blk, v_blk, block_size, scale=0.0, kernel=KERNEL_AUTO,
+                            want_lse=False):
+    B, N, Hq, D = q.shape
+    Hkv = k_ctx.shape[1]
+    dev = q.device.index if q.device.index is not None else torch.cuda.current_device()
+    key = ("bc", B, N, block_size, Hq, Hkv, D, float(scale), kernel, dev)
+    plan = _cached_plan(key, batch=B, q_heads=Hq, kv_heads=Hkv, head_dim=D, block=block_size, seq_len=N,
+                        scale=scale, kernel=kernel, device=dev)
+    return plan.block_attn_block_causal(q, k_ctx, v_ctx, k_blk, v_blk, want_lse=want_lse)
+
+
+def selftest_wait_timeout(device=0, timeout_us=20000, stream=None) -> int:
+    return lib().tt_selftest_wait_timeout(int(device), int(timeout_us), _stream(stream))
+
+
+def work_split(tiles_per_unit, num_ctas):
+    """Host-only: the library's range split for the given per-unit tile counts."""
+    n = len(tiles_per_unit)
+    tiles = (ctypes.c_int * max(n, 1))(*tiles_per_unit)
+    starts = (ctypes.c_longlong * (num_ctas + 1))()
+    first = (ctypes.c_int * max(n, 1))()
+    last = (ctypes.c_int * max(n, 1))()
+    _check(lib().tt_debug_work_split(n, tiles, num_ctas, starts, first, last), "tt_debug_work_split")
+    return list(starts), list(first)[:n], list(last)[:n]
