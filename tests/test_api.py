@@ -76,7 +76,7 @@ def test_null_arguments():
 
 
 @pytest.mark.parametrize("tiles,C", [
-    ([3, 5, 1, 7], 4), ([1] * 17, 5), ([40], 148), ([2, 2], 7), ([33] * 16, 148),
+    ([3, 5, 1, 7], 4), ([1] * 17, 5), ([40], 148), ([2, 2], 7), ([33] * 16, 148), ([5], 592),
     (list(np.random.default_rng(0).integers(1, 130, 128)), 148), ([1], 1),
 ])
 def test_work_split_partition(tiles, C):
@@ -85,9 +85,12 @@ def test_work_split_partition(tiles, C):
     bounds the partial slots at two per range."""
     starts, first, last = ops.work_split([int(t) for t in tiles], C)
     T = int(sum(tiles))
+    Ce = min(C, T)
     assert starts[0] == 0 and starts[-1] == T
     sizes = np.diff(starts)
-    assert sizes.min() >= T // C and sizes.max() <= -(-T // C)
+    # the first min(C, T) ranges are non-empty and near-equal; the rest are empty
+    assert sizes[:Ce].min() >= max(1, T // Ce) and sizes[:Ce].max() <= -(-T // Ce)
+    assert not sizes[Ce:].any()
     Tu = np.concatenate([[0], np.cumsum(tiles)])
     for u in range(len(tiles)):
         # brute force: ranges whose [start, end) meets [Tu, Tu + tiles)

@@ -527,11 +527,12 @@ tt_status_t tt_debug_work_split(int num_units, const int* tiles_per_unit, int nu
     if (tiles_per_unit[u] < 1) return fail(TT_ERR_INVALID_ARG, "every unit has at least one tile");
     T += tiles_per_unit[u];
   }
-  for (int c = 0; c <= num_ctas; ++c) range_start[c] = tt::range_start(T, num_ctas, c);
+  const int Ce = tt::used_ranges(T, num_ctas);
+  for (int c = 0; c <= num_ctas; ++c) range_start[c] = c <= Ce ? tt::range_start(T, Ce, c) : T;
   long long Tu = 0;
   for (int u = 0; u < num_units; ++u) {
-    unit_first[u] = tt::range_of_tile(T, num_ctas, Tu);
-    unit_last[u] = tt::range_of_tile(T, num_ctas, Tu + tiles_per_unit[u] - 1);
+    unit_first[u] = tt::range_of_tile(T, Ce, Tu);
+    unit_last[u] = tt::range_of_tile(T, Ce, Tu + tiles_per_unit[u] - 1);
     Tu += tiles_per_unit[u];
   }
   return TT_OK;

@@ -1,6 +1,482 @@
-// placeholder until the tcgen05 kernel lands
+// Block attention on the 5th-generation tensor cores (tcgen05 + TMEM + TMA).
+//
+// The method (paperfeed.app review of arXiv 2606.26493, "Nemotron-Labs-
+// TwoTower", section "The idea: freeze the reader, train the writer"): the S
+// noisy block queries of denoiser layer i attend, in one softmax, to the
+// frozen context tower's layer-i cache followed by the block's own keys.
+//
+// One persistent CTA per SM walks its range of key tiles (sched.cuh).  The
+// S*g query rows of a unit (all g query heads that share a KV head, for all S
+// block tokens) are packed into one or two 128-row tensor-core tiles, so each
+// key tile is read from HBM once and feeds up to 256 query rows.
+//
+// Roles (384 threads):
+//   warp 0       TMA producer: Q of each segment, then K and V tiles of every
+//                key tile into a ring of shared-memory slots (128-byte swizzle);
+//                for a tile whose valid rows are not a multiple of 16 it zeroes
+//                the V rows the last MMA k-step would otherwise read.
+//   warp 1       TMEM owner and MMA issuer (one thread): S_m = Q_m K^T into
+//                TMEM, O_m += P_m V with P read from TMEM (aliasing S_m).
+//   warps 4..7   softmax warpgroup of M-tile 0 (thread = TMEM lane = row)
+//   warps 8..11  softmax warpgroup of M-tile 1
+// TMEM columns: S_0 [0,128), S_1 [128,256), O_0 [256,256+D), O_1 [256+D, 256+2D).
+//
+// The softmax keeps a running reference maximum per row and rescales O (in
+// TMEM) only when a new maximum exceeds it by more than 2^8; the final
+// normalisation divides by the sum taken against the same reference, so the
+// result is exact up to rounding.
+//
+// Every wait is bounded (ptx.cuh: mbar_wait); on a timeout the CTA raises the
+// error word, drains what it issued, frees TMEM and returns.
 #include "problem.h"
+#include "ptx.cuh"
+#include "walker.cuh"
+
 namespace tt {
-size_t attn_tcgen05_smem_bytes(int) { return 0; }
-cudaError_t launch_attn_tcgen05(const Problem&, const TmaMaps&, cudaStream_t) { return cudaErrorNotSupported; }
+namespace {
+
+constexpr int kThreads = 384;
+constexpr int kKeyTile = 128;
+constexpr int kMaxRows = 256;
+constexpr int kRowBytes = 128;              // one 64-element bf16 row of a swizzled half
+constexpr float kRescaleThreshold = 8.0f;   // log2 units
+
+template <int D>
+struct Cfg {
+  static constexpr int kHalves = D / 64;
+  static constexpr int kStages = D == 128 ? 4 : 8;
+  static constexpr int kQBytes = kMaxRows * kRowBytes * kHalves;
+  static constexpr int kSlotBytes = kKeyTile * kRowBytes * kHalves;
+  static constexpr int kStageOff = kQBytes;
+  static constexpr int kEpiOff = kStageOff + kStages * kSlotBytes;
+  static constexpr int kEpiBytes = 8 * 32 * 32 * 4;  // 8 softmax warps x 32 rows x 32 fp32
+  static constexpr int kBarOff = kEpiOff + kEpiBytes;
+  static constexpr int kSmemBytes = kBarOff + 512 + 1024;  // barriers/flags + alignment slack
+};
+
+struct Bars {
+  uint64_t q_full, q_empty, tail, drain;
+  uint64_t s_full[2], p_full[2], o_full[2], o_empty[2];
+  uint64_t kv_full[8], kv_empty[8];
+};
+
+struct Shared {
+  uint32_t tmem_base;
+  int abort_flag;
+  long long T, start, end;
+  Unit first;
+};
+
+__device__ __forceinline__ int round16(int x) { return (x + 15) & ~15; }
+
+// Output row pointer of packed row r of unit x (final output or segment partial).
+__device__ __forceinline__ float* out_row(const Problem& p, const Unit& x, const Segment& sg, int r, int D) {
+  if (sg.full) {
+    const int t = r / p.g, j = r - (r / p.g) * p.g;
+    return p.out + ((size_t)(x.ns * p.S + t) * p.Hq + x.h * p.g + j) * D;
+  }
+  return p.part_o + ((size_t)sg.slot * p.R + r) * D;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_tcgen05_kernel(const Problem p, const __grid_constant__ TmaMaps maps) {
+  using C = Cfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t q_s = sbase;
+  const uint32_t kv_s = sbase + C::kStageOff;
+  float* epi = reinterpret_cast<float*>(smem + C::kEpiOff);
+  Bars* bars = reinterpret_cast<Bars*>(smem + C::kBarOff);
+  Shared* sh = reinterpret_cast<Shared*>(smem + C::kBarOff + sizeof(Bars));
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int c = blockIdx.x;
+  const int MT = p.R > 128 ? 2 : 1;
+
+  // ---------------------------------------------------------------- setup --
+  {
+    // zero Q (rows >= R stay zero for every segment) through the generic proxy
+    uint4* z = reinterpret_cast<uint4*>(smem);
+    for (int i = tid; i < C::kQBytes / 16; i += kThreads) z[i] = make_uint4(0, 0, 0, 0);
+    fence_proxy_async_smem();
+  }
+  if (tid == 0) {
+    mbar_init(smem_u32(&bars->q_full), 1);
+    mbar_init(smem_u32(&bars->q_empty), 1);
+    mbar_init(smem_u32(&bars->tail), 1);
+    mbar_init(smem_u32(&bars->drain), 1);
+    for (int m = 0; m < 2; ++m) {
+      mbar_init(smem_u32(&bars->s_full[m]), 1);
+      mbar_init(smem_u32(&bars->p_full[m]), 128);
+      mbar_init(smem_u32(&bars->o_full[m]), 1);
+      mbar_init(smem_u32(&bars->o_empty[m]), 128);
+    }
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(smem_u32(&bars->kv_full[s]), 1);
+      mbar_init(smem_u32(&bars->kv_empty[s]), 1);
+    }
+    sh->abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&maps.q);
+    tma_prefetch_desc(&maps.k_ctx);
+    tma_prefetch_desc(&maps.v_ctx);
+    tma_prefetch_desc(&maps.k_blk);
+    tma_prefetch_desc(&maps.v_blk);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&sh->tmem_base), 512);
+    tmem_relinquish();
+  }
+  if (warp == 2) {
+    long long T = 0, start = 0, end = 0;
+    Unit first;
+    find_range(p, c, T, start, end, first);
+    if (lane == 0) {
+      sh->T = T;
+      sh->start = start;
+      sh->end = end;
+      if (start < end) sh->first = first;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  const uint32_t tmem = sh->tmem_base;
+  const long long T = sh->T, start = sh->start, end = sh->end;
+  const WaitCtx wc{&sh->abort_flag, p.err_word, p.wait_limit_ns};
+  const bool have_work = start < end;
+
+  if (warp == 0 && have_work) {
+    // ============================================================ producer ==
+    uint32_t it = 0, q_it = 0, tail_ph = 0;
+    bool ok = true;
+    Unit x = sh->first;
+    for (; ok;) {
+      const Segment sg = segment_of(x, start, end, c);
+      ok = mbar_wait(smem_u32(&bars->q_empty), (q_it & 1) ^ 1, wc);
+      if (!ok) break;
+      if (lane == 0) {
+        const uint32_t bar = smem_u32(&bars->q_full);
+        mbar_arrive_expect_tx(bar, (uint32_t)(p.R * kRowBytes * C::kHalves));
+        for (int hf = 0; hf < C::kHalves; ++hf)
+          tma_load_3d(q_s + hf * (kMaxRows * kRowBytes), &maps.q, bar, hf * 64, x.h * p.g, x.ns * p.S);
+      }
+      ++q_it;
+      const int ctx_row0 = (x.n * p.Hkv + x.h) * p.ctx_stride;
+      for (int i = sg.lo; i < sg.hi && ok; ++i) {
+        const TileKeys tk = tile_keys(p, x, i);
+        const int box_rows = tk.is_blk ? min(p.S, kKeyTile) : kKeyTile;
+        const uint32_t bytes = (uint32_t)(box_rows * kRowBytes * C::kHalves);
+        for (int kv = 0; kv < 2 && ok; ++kv, ++it) {
+          const int s = it % C::kStages;
+          ok = mbar_wait(smem_u32(&bars->kv_empty[s]), ((it / C::kStages) & 1) ^ 1, wc);
+          if (!ok) break;
+          const uint32_t slot = kv_s + s * C::kSlotBytes;
+          const CUtensorMap* m = tk.is_blk ? (kv ? &maps.v_blk : &maps.k_blk) : (kv ? &maps.v_ctx : &maps.k_ctx);
+          // V rows [count, round16(count)) are read by the last PV k-step: zero them.
+          const bool fix = kv == 1 && (tk.count & 15) != 0;
+          const uint32_t bar = fix ? smem_u32(&bars->tail) : smem_u32(&bars->kv_full[s]);
+          if (lane == 0) {
+            mbar_arrive_expect_tx(bar, bytes);
+            for (int hf = 0; hf < C::kHalves; ++hf) {
+              const uint32_t dst = slot + hf * (kKeyTile * kRowBytes);
+              if (tk.is_blk) tma_load_3d(dst, m, bar, hf * 64, x.h, x.ns * p.S + tk.first);
+              else tma_load_2d(dst, m, bar, hf * 64, ctx_row0 + tk.first);
+            }
+          }
+          if (fix) {
+            ok = mbar_wait(smem_u32(&bars->tail), tail_ph, wc);
+            tail_ph ^= 1;
+            if (!ok) break;
+            const int r0 = tk.count, r1 = round16(tk.count);
+            const int n16 = (r1 - r0) * 8 * C::kHalves;  // 16-byte chunks to clear
+            for (int e = lane; e < n16; e += 32) {
+              const int hf = e / ((r1 - r0) * 8);
+              const int rem = e - hf * (r1 - r0) * 8;
+              const int row = r0 + rem / 8, ch = rem % 8;
+              uint4* dst = reinterpret_cast<uint4*>(smem + C::kStageOff + s * C::kSlotBytes +
+                                                    hf * (kKeyTile * kRowBytes) + row * kRowBytes + ch * 16);
+              *dst = make_uint4(0, 0, 0, 0);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&bars->kv_full[s]));
+          }
+        }
+      }
+      if (!ok || sg.last) break;
+      x = make_unit(p, x.u + 1, x.Tu + x.tiles);
+    }
+    if (!ok) {
+      // drain: wait (briefly) for loads that may still be landing in shared memory
+      WaitCtx dw{&sh->abort_flag, nullptr, 2000000ull};
+      int dummy = 0;
+      dw.abort_flag = &dummy;
+      for (uint32_t j = (it > (uint32_t)C::kStages ? it - C::kStages : 0); j < it; ++j)
+        mbar_wait(smem_u32(&bars->kv_full[j % C::kStages]), (j / C::kStages) & 1, dw);
+      if (q_it) mbar_wait(smem_u32(&bars->q_full), (q_it - 1) & 1, dw);
+    }
+  } else if (warp == 1 && have_work) {
+    // ============================================================= MMA warp ==
+    if (lane == 0) {
+      uint32_t it = 0, q_it = 0, t_cnt = 0, seg_cnt = 0;
+      bool ok = true;
+      Unit x = sh->first;
+      const uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
+      for (; ok;) {
+        const Segment sg = segment_of(x, start, end, c);
+        ok = mbar_wait(smem_u32(&bars->q_full), q_it & 1, wc);
+        ++q_it;
+        if (!ok) break;
+        tc_fence_after();
+        // S_m(i) = Q_m K_i^T
+        auto issue_s = [&](int m, uint32_t kslot, int n_mma) {
+          const uint32_t idesc = idesc_bf16_f32(128, n_mma, 0, 0);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const int hf = kk >> 2, ko = (kk & 3) * 32;
+            const uint64_t a = smem_desc_sw128(q_s + hf * (kMaxRows * kRowBytes) + m * 128 * kRowBytes + ko, 16, 1024);
+            const uint64_t b = smem_desc_sw128(kslot + hf * (kKeyTile * kRowBytes) + ko, 16, 1024);
+            tc_mma_ss(tmem + m * 128, a, b, idesc, kk > 0);
+          }
+        };
+        // prologue: S of the first tile
+        {
+          const int n0 = round16(tile_keys(p, x, sg.lo).count);
+          const int s = it % C::kStages;
+          ok = mbar_wait(smem_u32(&bars->kv_full[s]), (it / C::kStages) & 1, wc);
+          if (!ok) break;
+          tc_fence_after();
+          for (int m = 0; m < MT; ++m) {
+            issue_s(m, kv_s + s * C::kSlotBytes, n0);
+            tc_commit(smem_u32(&bars->s_full[m]));
+          }
+          tc_commit(smem_u32(&bars->kv_empty[s]));
+        }
+        for (int i = sg.lo; i < sg.hi && ok; ++i, ++t_cnt) {
+          const int nv = round16(tile_keys(p, x, i).count);
+          const int sv = (it + 1) % C::kStages;
+          ok = mbar_wait(smem_u32(&bars->kv_full[sv]), ((it + 1) / C::kStages) & 1, wc);
+          if (!ok) break;
+          const bool more = i + 1 < sg.hi;
+          const int sk2 = (it + 2) % C::kStages;
+          const int nn = more ? round16(tile_keys(p, x, i + 1).count) : 0;
+          for (int m = 0; m < MT && ok; ++m) {
+            ok = mbar_wait(smem_u32(&bars->p_full[m]), t_cnt & 1, wc);
+            if (ok && i == sg.lo) ok = mbar_wait(smem_u32(&bars->o_empty[m]), (seg_cnt & 1) ^ 1, wc);
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t vslot = kv_s + sv * C::kSlotBytes;
+            for (int kk = 0; kk < nv / 16; ++kk) {
+              const uint64_t b = smem_desc_sw128(vslot + kk * 16 * kRowBytes, kKeyTile * kRowBytes, 1024);
+              tc_mma_ts(tmem + 256 + m * D, tmem + m * 128 + kk * 8, b, idesc_pv, (i > sg.lo || kk > 0) ? 1u : 0u);
+            }
+            if (more) {
+              if (m == 0) {
+                ok = mbar_wait(smem_u32(&bars->kv_full[sk2]), ((it + 2) / C::kStages) & 1, wc);
+                if (!ok) break;
+                tc_fence_after();
+              }
+              issue_s(m, kv_s + sk2 * C::kSlotBytes, nn);
+              tc_commit(smem_u32(&bars->s_full[m]));
+            }
+          }
+          if (!ok) break;
+          tc_commit(smem_u32(&bars->kv_empty[sv]));
+          if (more) tc_commit(smem_u32(&bars->kv_empty[sk2]));
+          it += 2;
+        }
+        if (!ok) break;
+        for (int m = 0; m < MT; ++m) tc_commit(smem_u32(&bars->o_full[m]));
+        tc_commit(smem_u32(&bars->q_empty));
+        ++seg_cnt;
+        if (sg.last) break;
+        x = make_unit(p, x.u + 1, x.Tu + x.tiles);
+      }
+      // drain every MMA this thread issued before TMEM can be released
+      tc_commit(smem_u32(&bars->drain));
+      int dummy = 0;
+      WaitCtx dw{&dummy, nullptr, 2000000ull};
+      mbar_wait(smem_u32(&bars->drain), 0, dw);
+    }
+    __syncwarp();
+  } else if (warp >= 4 && have_work) {
+    // ========================================================= softmax WGs ==
+    const int m = (warp - 4) >> 2;
+    const int q4 = warp & 3;             // TMEM lane quarter of this warp
+    const int row = q4 * 32 + lane;      // row within the M-tile
+    const int r = m * 128 + row;         // packed row of the unit
+    if (m < MT) {
+      const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+      const uint32_t s_addr = tmem + lane_off + m * 128;
+      const uint32_t o_addr = tmem + lane_off + 256 + m * D;
+      float* stage = epi + (warp - 4) * 32 * 32;
+      uint32_t t_cnt = 0, seg_cnt = 0;
+      bool ok = true;
+      Unit x = sh->first;
+      for (; ok;) {
+        const Segment sg = segment_of(x, start, end, c);
+        float m_ref = -INFINITY, l = 0.f;
+        for (int i = sg.lo; i < sg.hi; ++i, ++t_cnt) {
+          const int count = tile_keys(p, x, i).count;
+          ok = mbar_wait(smem_u32(&bars->s_full[m]), t_cnt & 1, wc);
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            const int cbase = half * 64;
+            if (cbase >= count) break;  // uniform: the tile has no keys here
+            uint32_t v[64];
+            tmem_ld32(s_addr + cbase, v);
+            if (cbase + 32 < count) tmem_ld32(s_addr + cbase + 32, v + 32);
+            tc_wait_ld();
+            float mx = -INFINITY;
+#pragma unroll
+            for (int k = 0; k < 64; ++k) {
+              const float sv = cbase + k < count ? __uint_as_float(v[k]) * p.scale_log2 : -INFINITY;
+              v[k] = __float_as_uint(sv);
+              mx = fmaxf(mx, sv);
+            }
+            if (i == sg.lo && half == 0) {
+              m_ref = mx;  // O is overwritten by the first PV of the segment
+            } else {
+              const bool need = mx > m_ref + kRescaleThreshold;
+              const float alpha = need ? fast_exp2(m_ref - mx) : 1.f;
+              if (need) {
+                m_ref = mx;
+                l *= alpha;
+              }
+              // O holds this segment's sum only after its first PV: rescale from tile 2 on
+              if (i > sg.lo && __any_sync(0xffffffffu, need)) {
+#pragma unroll 1
+                for (int cc = 0; cc < D / 16; ++cc) {
+                  uint32_t o[16];
+                  tmem_ld16(o_addr + cc * 16, o);
+                  tc_wait_ld();
+#pragma unroll
+                  for (int k = 0; k < 16; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+                  tmem_st16(o_addr + cc * 16, o);
+                }
+              }
+            }
+            float sum = 0.f;
+#pragma unroll
+            for (int ch = 0; ch < 2; ++ch) {
+              if (cbase + 32 * ch >= count) break;
+              uint32_t pk[16];
+#pragma unroll
+              for (int k = 0; k < 16; ++k) {
+                const float a = fast_exp2(__uint_as_float(v[32 * ch + 2 * k]) - m_ref);
+                const float b = fast_exp2(__uint_as_float(v[32 * ch + 2 * k + 1]) - m_ref);
+                sum += a + b;
+                pk[k] = pack_bf16(a, b);
+              }
+              // P as bf16 pairs over the first half of this S chunk's columns
+              tmem_st16(s_addr + (cbase >> 1) + 16 * ch, pk);
+            }
+            l += sum;
+          }
+          if (!ok) break;
+          tc_wait_st();
+          tc_fence_before();
+          mbar_arrive(smem_u32(&bars->p_full[m]));
+        }
+        if (!ok) break;
+        // ---- epilogue: O / l to the output (or the segment's partial) ----
+        ok = mbar_wait(smem_u32(&bars->o_full[m]), seg_cnt & 1, wc);
+        if (!ok) break;
+        tc_fence_after();
+        const float inv = 1.f / l;
+        const int rbase = m * 128 + q4 * 32;  // first packed row of this warp
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t o[32];
+          tmem_ld32(o_addr + cc * 32, o);
+          tc_wait_ld();
+          if (cc == D / 32 - 1) {
+            tc_fence_before();
+            mbar_arrive(smem_u32(&bars->o_empty[m]));  // O fully read: the next segment may overwrite it
+          }
+          // stage the 32x32 block (16-byte chunks XOR-swizzled by row) for coalesced stores
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            float4 f = make_float4(__uint_as_float(o[4 * q]) * inv, __uint_as_float(o[4 * q + 1]) * inv,
+                                   __uint_as_float(o[4 * q + 2]) * inv, __uint_as_float(o[4 * q + 3]) * inv);
+            reinterpret_cast<float4*>(stage + lane * 32)[q ^ (lane & 7)] = f;
+          }
+          __syncwarp();
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const int rr = k * 4 + (lane >> 3);  // row within the warp's 32
+            const int q = lane & 7;
+            const int gr = rbase + rr;
+            if (gr < p.R) {
+              float4 f = reinterpret_cast<const float4*>(stage + rr * 32)[q ^ (rr & 7)];
+              float* dst = out_row(p, x, sg, gr, D) + cc * 32 + q * 4;
+              *reinterpret_cast<float4*>(dst) = f;
+            }
+          }
+          __syncwarp();
+        }
+        if (r < p.R) {
+          const float lse = (m_ref + __log2f(l)) * 0.6931471805599453f;
+          if (sg.full) {
+            if (p.lse) {
+              const int t = r / p.g, j = r - (r / p.g) * p.g;
+              p.lse[(size_t)(x.n * p.Hq + x.h * p.g + j) * (p.NB * p.S) + x.b * p.S + t] = lse;
+            }
+          } else {
+            p.part_lse[(size_t)sg.slot * p.R + r] = lse;
+          }
+        }
+        ++seg_cnt;
+        if (sg.last) break;
+        x = make_unit(p, x.u + 1, x.Tu + x.tiles);
+      }
+    }
+  }
+
+  // record for the combine: the cut unit (if any) that begins in this range
+  if (tid == 64) {
+    SplitRecord rec{-1, -1, 0, 0};
+    if (have_work) {
+      Unit x = sh->first;
+      while (x.Tu + x.tiles < end) x = make_unit(p, x.u + 1, x.Tu + x.tiles);
+      rec = record_of(x, T, p.C, start, end);
+    }
+    p.records[c] = rec;
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+}  // namespace
+
+size_t attn_tcgen05_smem_bytes(int D) {
+  return D == 128 ? (size_t)Cfg<128>::kSmemBytes : (size_t)Cfg<64>::kSmemBytes;
+}
+
+cudaError_t launch_attn_tcgen05(const Problem& p, const TmaMaps& maps, cudaStream_t stream) {
+  static const bool attr_done = [] {
+    cudaFuncSetAttribute(attn_tcgen05_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         Cfg<128>::kSmemBytes);
+    cudaFuncSetAttribute(attn_tcgen05_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         Cfg<64>::kSmemBytes);
+    return true;
+  }();
+  (void)attr_done;
+  if (p.D == 128)
+    attn_tcgen05_kernel<128><<<p.C, kThreads, Cfg<128>::kSmemBytes, stream>>>(p, maps);
+  else
+    attn_tcgen05_kernel<64><<<p.C, kThreads, Cfg<64>::kSmemBytes, stream>>>(p, maps);
+  return cudaGetLastError();
+}
+
 }  // namespace tt

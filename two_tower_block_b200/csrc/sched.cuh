@@ -4,8 +4,8 @@
 // rows attend to one key list.  Its key list is cut into tiles: tile 0 is the
 // block's own S keys, tiles 1.. are the visible context keys, key_tile at a
 // time.  All units' tiles are laid end to end (unit-major) into one global
-// sequence of T tiles, and range c of C gets tiles [floor(c*T/C),
-// floor((c+1)*T/C)).  Every range therefore carries the same work up to one
+// sequence of T tiles, and range c of C' = min(C, T) gets tiles [floor(c*T/C'),
+// floor((c+1)*T/C')); ranges c >= C' are empty.  Every range therefore carries the same work up to one
 // tile, whatever the length mix, and a unit is cut only where a range
 // boundary falls inside it.
 //
@@ -27,6 +27,10 @@
 namespace tt {
 
 TT_HD long long range_start(long long T, int C, int c) { return (long long)c * T / C; }
+
+// Ranges actually used: min(C, T), so that every used range holds at least one
+// tile and the ranges touching a cut unit are consecutive and all non-empty.
+TT_HD int used_ranges(long long T, int C) { return T < (long long)C ? (int)T : C; }
 
 // Index of the range whose [start, end) contains global tile x (0 <= x < T):
 // the largest c with floor(c*T/C) <= x, i.e. ceil((x+1)*C/T) - 1.

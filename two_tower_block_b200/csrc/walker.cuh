@@ -72,9 +72,13 @@ __device__ __forceinline__ void find_range(const Problem& p, int c, long long& T
   } else {
     T = p.T_causal;
   }
-  start = range_start(T, p.C, c);
-  end = range_start(T, p.C, c + 1);
-  if (start >= end) return;
+  const int Ce = used_ranges(T, p.C);
+  if (c >= Ce) {
+    start = end = T;
+    return;
+  }
+  start = range_start(T, Ce, c);
+  end = range_start(T, Ce, c + 1);
   if (p.mode == kDecode) {
     long long acc = 0;
     for (int base = 0; base < p.B; base += 32) {
@@ -134,8 +138,10 @@ __device__ __forceinline__ Segment segment_of(const Unit& x, long long start, lo
 }
 
 // The record of range c: the cut unit that begins in c and runs past its end.
+// C is the plan's range count; the split uses min(C, T) of them.
 __device__ __forceinline__ SplitRecord record_of(const Unit& last, long long T, int C, long long start,
                                                  long long end) {
+  C = used_ranges(T, C);
   SplitRecord r;
   r.unit = -1;
   r.last_range = -1;
