@@ -158,8 +158,8 @@ TT_API tt_status_t tt_block_attn_check(tt_plan_t plan, tt_stream_t stream);
  * bracketed by two CUDA events recorded on the launching stream (up to 4096
  * launches are kept).  tt_block_attn_profile_read synchronises on the recorded
  * events and returns, for kernel id 0 (attention) or 1 (split combine), the
- * number of launches and their summed duration in milliseconds, then clears
- * the record. */
+ * number of launches and their summed duration in milliseconds.  Calling
+ * tt_block_attn_profile again clears the record. */
 TT_API tt_status_t tt_block_attn_profile(tt_plan_t plan, int enable);
 TT_API tt_status_t tt_block_attn_profile_read(tt_plan_t plan, int kernel_id, int* launches, double* total_ms);
 

@@ -494,7 +494,6 @@ tt_status_t tt_block_attn_profile_read(tt_plan_t plan, int kernel_id, int* launc
   }
   *launches = n;
   *total_ms = tot;
-  plan->prof_n = 0;
   return TT_OK;
 }
 

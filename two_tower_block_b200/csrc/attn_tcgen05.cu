@@ -327,60 +327,62 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = mbar_wait(smem_u32(&bars->s_full[m]), t_cnt & 1, wc);
           if (!ok) break;
           tc_fence_after();
+          // pass 1: row maximum of this tile (masked beyond `count`), log2 units
+          float mx = -INFINITY;
 #pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            const int cbase = half * 64;
-            if (cbase >= count) break;  // uniform: the tile has no keys here
+          for (int ch = 0; ch < kKeyTile / 32; ch += 2) {
+            if (32 * ch >= count) break;
             uint32_t v[64];
-            tmem_ld32(s_addr + cbase, v);
-            if (cbase + 32 < count) tmem_ld32(s_addr + cbase + 32, v + 32);
+            tmem_ld32(s_addr + 32 * ch, v);
+            if (32 * ch + 32 < count) tmem_ld32(s_addr + 32 * ch + 32, v + 32);
             tc_wait_ld();
-            float mx = -INFINITY;
 #pragma unroll
-            for (int k = 0; k < 64; ++k) {
-              const float sv = cbase + k < count ? __uint_as_float(v[k]) * p.scale_log2 : -INFINITY;
-              v[k] = __float_as_uint(sv);
-              mx = fmaxf(mx, sv);
-            }
-            if (i == sg.lo && half == 0) {
-              m_ref = mx;  // O is overwritten by the first PV of the segment
-            } else {
-              const bool need = mx > m_ref + kRescaleThreshold;
+            for (int k = 0; k < 64; ++k)
+              mx = fmaxf(mx, 32 * ch + k < count ? __uint_as_float(v[k]) : -INFINITY);
+          }
+          mx *= p.scale_log2;
+          if (i == sg.lo) {
+            m_ref = mx;  // O is overwritten by the first PV of the segment
+          } else {
+            const bool need = mx > m_ref + kRescaleThreshold;
+            if (__any_sync(0xffffffffu, need)) {
               const float alpha = need ? fast_exp2(m_ref - mx) : 1.f;
               if (need) {
                 m_ref = mx;
                 l *= alpha;
               }
-              // O holds this segment's sum only after its first PV: rescale from tile 2 on
-              if (i > sg.lo && __any_sync(0xffffffffu, need)) {
 #pragma unroll 1
-                for (int cc = 0; cc < D / 16; ++cc) {
-                  uint32_t o[16];
-                  tmem_ld16(o_addr + cc * 16, o);
-                  tc_wait_ld();
+              for (int cc = 0; cc < D / 16; ++cc) {
+                uint32_t o[16];
+                tmem_ld16(o_addr + cc * 16, o);
+                tc_wait_ld();
 #pragma unroll
-                  for (int k = 0; k < 16; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
-                  tmem_st16(o_addr + cc * 16, o);
-                }
+                for (int k = 0; k < 16; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+                tmem_st16(o_addr + cc * 16, o);
               }
             }
-            float sum = 0.f;
-#pragma unroll
-            for (int ch = 0; ch < 2; ++ch) {
-              if (cbase + 32 * ch >= count) break;
-              uint32_t pk[16];
-#pragma unroll
-              for (int k = 0; k < 16; ++k) {
-                const float a = fast_exp2(__uint_as_float(v[32 * ch + 2 * k]) - m_ref);
-                const float b = fast_exp2(__uint_as_float(v[32 * ch + 2 * k + 1]) - m_ref);
-                sum += a + b;
-                pk[k] = pack_bf16(a, b);
-              }
-              // P as bf16 pairs over the first half of this S chunk's columns
-              tmem_st16(s_addr + (cbase >> 1) + 16 * ch, pk);
-            }
-            l += sum;
           }
+          // pass 2: p = 2^(s - m_ref), row sum, P as bf16 pairs over S's first columns
+          // (keys [32ch, 32ch+32) -> columns [16ch, 16ch+16); chunk ch's S is read first)
+          float sum = 0.f;
+#pragma unroll
+          for (int ch = 0; ch < kKeyTile / 32; ++ch) {
+            if (32 * ch >= count) break;
+            uint32_t v[32];
+            tmem_ld32(s_addr + 32 * ch, v);
+            tc_wait_ld();
+            uint32_t pk[16];
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+              const int c0 = 32 * ch + 2 * k;
+              const float a = c0 < count ? fast_exp2(fmaf(__uint_as_float(v[2 * k]), p.scale_log2, -m_ref)) : 0.f;
+              const float b = c0 + 1 < count ? fast_exp2(fmaf(__uint_as_float(v[2 * k + 1]), p.scale_log2, -m_ref)) : 0.f;
+              sum += a + b;
+              pk[k] = pack_bf16(a, b);
+            }
+            tmem_st16(s_addr + 16 * ch, pk);
+          }
+          l += sum;
           if (!ok) break;
           tc_wait_st();
           tc_fence_before();
