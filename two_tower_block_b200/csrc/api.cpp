@@ -254,7 +254,7 @@ tt_status_t tt_block_attn_plan(const tt_block_attn_desc* desc, int device, tt_pl
   P->g = g;
   P->R = d.block_size * g;
   P->scale = d.scale > 0.f ? d.scale : 1.0f / std::sqrt((float)d.head_dim);
-  P->kernel = d.kernel == TT_KERNEL_AUTO ? TT_KERNEL_MMA_SYNC : d.kernel;
+  P->kernel = d.kernel == TT_KERNEL_AUTO ? TT_KERNEL_TCGEN05 : d.kernel;
   if (P->kernel == TT_KERNEL_TCGEN05 && prop.major != 10) P->kernel = TT_KERNEL_MMA_SYNC;
   if (P->kernel == TT_KERNEL_TCGEN05) {
     P->key_tile = 128;
