@@ -149,6 +149,30 @@ TT_API tt_status_t tt_block_attn_host(tt_plan_t plan, const void* q, const void*
                                const void* k_blk, const void* v_blk, const int32_t* ctx_lens,
                                float* out, float* lse, tt_stream_t stream);
 
+/* Decode without any device allocation, for callers that cannot call cudaMalloc
+ * (engines and plugins that own all device memory and forbid further allocations,
+ * or serving loops that must never stall on an allocation).  The paper has no
+ * counterpart: this is a deployment variant of tt_block_attn.
+ *   desc      shape as for tt_block_attn_plan; seq_len and flags must be 0.
+ *             num_ctas = 0 picks the work split automatically; an explicit
+ *             num_ctas whose scratch exceeds the limit below is rejected with
+ *             TT_ERR_INVALID_ARG (tt_last_error_detail states the sizes).
+ *   q .. lse  exactly as for tt_block_attn (device memory, same layouts).
+ *   status    optional device uint32: zeroed, then receives the device error
+ *             bits (1 = ctx_lens out of range, 2 = a wait timed out); NULL
+ *             discards them.
+ * Scratch: one file-scope device array of 16 MiB that every GPU loading this
+ * library keeps until the process exits.  The first call on a device (with
+ * that device current) resolves the array's device address; make that first
+ * call before any stream capture.  Every call shares the array and leaves its
+ * contents behind, so calls that overlap on the GPU (different streams, or
+ * different host threads on one device) race: order them.  The call allocates
+ * nothing and does not synchronise. */
+TT_API tt_status_t tt_block_attn_noalloc(const tt_block_attn_desc* desc, const void* q, const void* k_ctx,
+                                         const void* v_ctx, const void* k_blk, const void* v_blk,
+                                         const int32_t* ctx_lens, float* out, float* lse, uint32_t* status,
+                                         tt_stream_t stream);
+
 /* Synchronise `stream`, then read and clear the plan's device error word.
  * Returns TT_OK, TT_ERR_DEVICE_ARG or TT_ERR_TIMEOUT (or TT_ERR_CUDA if the
  * synchronisation itself failed). */

@@ -16,9 +16,13 @@
 #include "errbits.h"
 #include "sched.cuh"
 
-namespace {
-
+// Detail text of the last host-side error on this thread (read by tt_last_error_detail).
+namespace tt {
 thread_local std::string g_detail;
+}
+using tt::g_detail;
+
+namespace {
 
 tt_status_t fail(tt_status_t st, const std::string& why) {
   g_detail = why;

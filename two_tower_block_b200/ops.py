@@ -31,7 +31,7 @@ EXPORTED_SYMBOLS = [
     "tt_block_attn_plan", "tt_block_attn_plan_destroy", "tt_block_attn_plan_get_info", "tt_block_attn",
     "tt_block_attn_block_causal", "tt_block_attn_host", "tt_block_attn_check", "tt_block_attn_profile",
     "tt_block_attn_profile_read", "tt_selftest_wait_timeout", "tt_debug_work_split", "tt_status_string",
-    "tt_last_error_detail",
+    "tt_last_error_detail", "tt_block_attn_noalloc",
 ]
 
 
@@ -72,6 +72,7 @@ def lib() -> ctypes.CDLL:
     L.tt_block_attn_profile_read.argtypes = [vp, i, ip, ctypes.POINTER(ctypes.c_double)]
     L.tt_selftest_wait_timeout.argtypes = [i, i, vp]
     L.tt_debug_work_split.argtypes = [i, ip, i, ctypes.POINTER(ctypes.c_longlong), ip, ip]
+    L.tt_block_attn_noalloc.argtypes = [ctypes.POINTER(Desc)] + [vp] * 10
     L.tt_status_string.argtypes = [i]
     L.tt_status_string.restype = ctypes.c_char_p
     L.tt_last_error_detail.argtypes = []
@@ -254,3 +255,16 @@ def work_split(tiles_per_unit, num_ctas):
     last = (ctypes.c_int * max(n, 1))()
     _check(lib().tt_debug_work_split(n, tiles, num_ctas, starts, first, last), "tt_debug_work_split")
     return list(starts), list(first)[:n], list(last)[:n]
+
+
+def block_attn_noalloc(q, k_ctx, v_ctx, k_blk, v_blk, ctx_lens, out, lse=None, status=None, scale=0.0,
+                       kernel=KERNEL_AUTO, num_ctas=0, stream=None):
+    """Decode through tt_block_attn_noalloc: no plan, no device allocation inside the
+    library (its scratch is a fixed 16 MiB device array).  Outputs are caller-owned;
+    `status` is an optional one-element uint32/int32 device tensor for the error bits."""
+    B, S, Hq, D = q.shape
+    Hkv, Lcap = k_ctx.shape[1], k_ctx.shape[2]
+    d = Desc(B, Hq, Hkv, D, S, Lcap, 0, float(scale), kernel, num_ctas, 0, 0)
+    return lib().tt_block_attn_noalloc(ctypes.byref(d), _ptr(q), _ptr(k_ctx), _ptr(v_ctx), _ptr(k_blk),
+                                       _ptr(v_blk), _ptr(ctx_lens), _ptr(out), _ptr(lse), _ptr(status),
+                                       _stream(stream))
