@@ -40,6 +40,11 @@ constexpr int kKeyTile = 128;
 constexpr int kMaxRows = 256;
 constexpr int kRowBytes = 128;              // one 64-element bf16 row of a swizzled half
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
+// Register split per warpgroup (launch: 168 per thread = 65536 / 384 rounded down to 8):
+// control warpgroup (warps 0-3) 4 x 32 x kCtrlRegs + softmax (warps 4-11) 8 x 32 x kSoftmaxRegs.
+constexpr int kCtrlRegs = 80;
+constexpr int kSoftmaxRegs = 200;
+static_assert(4 * 32 * kCtrlRegs + 8 * 32 * kSoftmaxRegs <= kThreads * 168, "register split exceeds the launch");
 
 template <int D>
 struct Cfg {
@@ -76,6 +81,48 @@ __device__ __forceinline__ float* out_row(const Problem& p, const Unit& x, const
     return p.out + ((size_t)(x.ns * p.S + t) * p.Hq + x.h * p.g + j) * D;
   }
   return p.part_o + ((size_t)sg.slot * p.R + r) * D;
+}
+
+// Row maximum of the first `count` raw scores of a tile (all kKeyTile when kFull).
+template <bool kFull>
+__device__ __forceinline__ float tile_row_max(const uint32_t* v, int count) {
+  float m[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+  for (int k = 0; k < kKeyTile; ++k) {
+    const float x = __uint_as_float(v[k]);
+    m[k & 3] = fmaxf(m[k & 3], (kFull || k < count) ? x : -INFINITY);
+  }
+  return fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
+}
+
+// p = 2^(s*c - m_ref) for the tile's keys (0 beyond `count`), written to TMEM as bf16
+// pairs over the first columns of the S region: keys [32ch, 32ch+32) -> columns
+// [16ch, 16ch+16).  Returns the row sum of p (fp32, before the bf16 rounding).
+template <bool kFull>
+__device__ __forceinline__ float tile_exp_store(const uint32_t* v, int count, float c, float m_ref,
+                                                uint32_t s_addr) {
+  const float2 c2 = make_float2(c, c);
+  const float2 nm2 = make_float2(-m_ref, -m_ref);
+  float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int ch = 0; ch < kKeyTile / 32; ++ch) {
+    if (!kFull && 32 * ch >= count) break;
+    uint32_t pk[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const int c0 = 32 * ch + 2 * k;
+      const float2 x = __ffma2_rn(make_float2(__uint_as_float(v[c0]), __uint_as_float(v[c0 + 1])), c2, nm2);
+      float a = fast_exp2(x.x), b = fast_exp2(x.y);
+      if (!kFull) {
+        a = c0 < count ? a : 0.f;
+        b = c0 + 1 < count ? b : 0.f;
+      }
+      acc = __fadd2_rn(acc, make_float2(a, b));
+      pk[k] = pack_bf16(a, b);
+    }
+    tmem_st16(s_addr + 16 * ch, pk);
+  }
+  return acc.x + acc.y;
 }
 
 template <int D>
@@ -151,6 +198,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const WaitCtx wc{&sh->abort_flag, p.err_word, p.wait_limit_ns};
   const bool have_work = start < end;
 
+  if (have_work && warp < 4) regs_dec<kCtrlRegs>();
   if (warp == 0 && have_work) {
     // ============================================================ producer ==
     uint32_t it = 0, q_it = 0, tail_ph = 0;
@@ -307,6 +355,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp >= 4 && have_work) {
     // ========================================================= softmax WGs ==
+    regs_inc<kSoftmaxRegs>();
     const int m = (warp - 4) >> 2;
     const int q4 = warp & 3;             // TMEM lane quarter of this warp
     const int row = q4 * 32 + lane;      // row within the M-tile
@@ -327,20 +376,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = mbar_wait(smem_u32(&bars->s_full[m]), t_cnt & 1, wc);
           if (!ok) break;
           tc_fence_after();
-          // pass 1: row maximum of this tile (masked beyond `count`), log2 units
-          float mx = -INFINITY;
+          // the tile's S row in registers; row maximum in log2 units (masked beyond `count`)
+          const bool full = count == kKeyTile;
+          uint32_t v[kKeyTile];
 #pragma unroll
-          for (int ch = 0; ch < kKeyTile / 32; ch += 2) {
-            if (32 * ch >= count) break;
-            uint32_t v[64];
-            tmem_ld32(s_addr + 32 * ch, v);
-            if (32 * ch + 32 < count) tmem_ld32(s_addr + 32 * ch + 32, v + 32);
-            tc_wait_ld();
-#pragma unroll
-            for (int k = 0; k < 64; ++k)
-              mx = fmaxf(mx, 32 * ch + k < count ? __uint_as_float(v[k]) : -INFINITY);
-          }
-          mx *= p.scale_log2;
+          for (int ch = 0; ch < kKeyTile / 32; ++ch)
+            if (full || 32 * ch < count) tmem_ld32(s_addr + 32 * ch, v + 32 * ch);
+          tc_wait_ld();
+          const float mx = (full ? tile_row_max<true>(v, count) : tile_row_max<false>(v, count)) * p.scale_log2;
           if (i == sg.lo) {
             m_ref = mx;  // O is overwritten by the first PV of the segment
           } else {
@@ -362,26 +405,8 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
             }
           }
-          // pass 2: p = 2^(s - m_ref), row sum, P as bf16 pairs over S's first columns
-          // (keys [32ch, 32ch+32) -> columns [16ch, 16ch+16); chunk ch's S is read first)
-          float sum = 0.f;
-#pragma unroll
-          for (int ch = 0; ch < kKeyTile / 32; ++ch) {
-            if (32 * ch >= count) break;
-            uint32_t v[32];
-            tmem_ld32(s_addr + 32 * ch, v);
-            tc_wait_ld();
-            uint32_t pk[16];
-#pragma unroll
-            for (int k = 0; k < 16; ++k) {
-              const int c0 = 32 * ch + 2 * k;
-              const float a = c0 < count ? fast_exp2(fmaf(__uint_as_float(v[2 * k]), p.scale_log2, -m_ref)) : 0.f;
-              const float b = c0 + 1 < count ? fast_exp2(fmaf(__uint_as_float(v[2 * k + 1]), p.scale_log2, -m_ref)) : 0.f;
-              sum += a + b;
-              pk[k] = pack_bf16(a, b);
-            }
-            tmem_st16(s_addr + 16 * ch, pk);
-          }
+          const float sum = full ? tile_exp_store<true>(v, count, p.scale_log2, m_ref, s_addr)
+                                 : tile_exp_store<false>(v, count, p.scale_log2, m_ref, s_addr);
           l += sum;
           if (!ok) break;
           tc_wait_st();

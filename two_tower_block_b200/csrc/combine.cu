@@ -12,8 +12,9 @@
 namespace tt {
 namespace {
 
-constexpr int kRowsPerBlock = 16;
+constexpr int kRowsPerBlock = 8;   // one warp per row
 constexpr int kThreads = 256;
+constexpr int kMaxSegInRegs = 32;  // segments whose weight one lane keeps (lane s holds segment s)
 
 template <int D>
 __global__ void __launch_bounds__(kThreads) combine_kernel(const Problem p) {
@@ -21,46 +22,67 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const Problem p) {
   const SplitRecord rec = p.records[c];
   if (rec.unit < 0) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r = blockIdx.y * kRowsPerBlock + warp;
+  if (r >= p.R) return;
   const Unit x = make_unit(p, rec.unit, 0);
   const int nseg = rec.last_range - c + 1;
   constexpr int V = D / 32;  // columns per lane
-  const int r_end = min(p.R, (int)(blockIdx.y + 1) * kRowsPerBlock);
-  for (int r = blockIdx.y * kRowsPerBlock + warp; r < r_end; r += kThreads / 32) {
-    float M = -INFINITY;
-    for (int s = lane; s < nseg; s += 32) {
-      const int slot = s == 0 ? 2 * c + rec.first_which : 2 * (c + s);
-      M = fmaxf(M, p.part_lse[(size_t)slot * p.R + r]);
-    }
+  auto slot_of = [&](int s) { return s == 0 ? 2 * c + rec.first_which : 2 * (c + s); };
+  // weights: lane s holds segment s (segments beyond 32 are folded in a second sweep)
+  float M = -INFINITY;
+  for (int s = lane; s < nseg; s += 32) M = fmaxf(M, p.part_lse[(size_t)slot_of(s) * p.R + r]);
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    float acc[V];
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  float acc[V];
 #pragma unroll
-    for (int v = 0; v < V; ++v) acc[v] = 0.f;
-    float wsum = 0.f;
-    for (int s = 0; s < nseg; ++s) {
-      const int slot = s == 0 ? 2 * c + rec.first_which : 2 * (c + s);
-      const float w = expf(p.part_lse[(size_t)slot * p.R + r] - M);
-      wsum += w;
-      const float* src = p.part_o + ((size_t)slot * p.R + r) * D + lane * V;
-      if constexpr (V == 4) {
-        const float4 a = *reinterpret_cast<const float4*>(src);
-        acc[0] += w * a.x; acc[1] += w * a.y; acc[2] += w * a.z; acc[3] += w * a.w;
-      } else {
-        const float2 a = *reinterpret_cast<const float2*>(src);
-        acc[0] += w * a.x; acc[1] += w * a.y;
+  for (int v = 0; v < V; ++v) acc[v] = 0.f;
+  float wsum = 0.f;
+  for (int s0 = 0; s0 < nseg; s0 += kMaxSegInRegs) {
+    const int s = s0 + lane;
+    const float w_lane = s < nseg ? expf(p.part_lse[(size_t)slot_of(s) * p.R + r] - M) : 0.f;
+    float ws = w_lane;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ws += __shfl_xor_sync(0xffffffffu, ws, o);
+    wsum += ws;
+    const int n = min(kMaxSegInRegs, nseg - s0);
+    // four segments' rows in flight per step
+    for (int k = 0; k < n; k += 4) {
+      float a[4][V];
+      float w[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        w[u] = __shfl_sync(0xffffffffu, w_lane, (k + u) & 31);
+        if (k + u < n) {
+          const float* src = p.part_o + ((size_t)slot_of(s0 + k + u) * p.R + r) * D + lane * V;
+          if constexpr (V == 4) {
+            const float4 t = __ldcg(reinterpret_cast<const float4*>(src));
+            a[u][0] = t.x; a[u][1] = t.y; a[u][2] = t.z; a[u][3] = t.w;
+          } else {
+            const float2 t = __ldcg(reinterpret_cast<const float2*>(src));
+            a[u][0] = t.x; a[u][1] = t.y;
+          }
+        } else {
+          w[u] = 0.f;
+#pragma unroll
+          for (int v = 0; v < V; ++v) a[u][v] = 0.f;
+        }
       }
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int v = 0; v < V; ++v) acc[v] = fmaf(w[u], a[u][v], acc[v]);
     }
-    const float inv = 1.f / wsum;
-    const int t = r / p.g, j = r - (r / p.g) * p.g;
-    float* dst = p.out + ((size_t)(x.ns * p.S + t) * p.Hq + x.h * p.g + j) * D + lane * V;
-    if constexpr (V == 4) {
-      *reinterpret_cast<float4*>(dst) = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
-    } else {
-      *reinterpret_cast<float2*>(dst) = make_float2(acc[0] * inv, acc[1] * inv);
-    }
-    if (lane == 0 && p.lse)
-      p.lse[(size_t)(x.n * p.Hq + x.h * p.g + j) * (p.NB * p.S) + x.b * p.S + t] = M + logf(wsum);
   }
+  const float inv = 1.f / wsum;
+  const int t = r / p.g, j = r - (r / p.g) * p.g;
+  float* dst = p.out + ((size_t)(x.ns * p.S + t) * p.Hq + x.h * p.g + j) * D + lane * V;
+  if constexpr (V == 4) {
+    *reinterpret_cast<float4*>(dst) = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+  } else {
+    *reinterpret_cast<float2*>(dst) = make_float2(acc[0] * inv, acc[1] * inv);
+  }
+  if (lane == 0 && p.lse)
+    p.lse[(size_t)(x.n * p.Hq + x.h * p.g + j) * (p.NB * p.S) + x.b * p.S + t] = M + logf(wsum);
 }
 
 // One thread waits on a barrier that nothing arrives at; the bounded wait must
