@@ -4,6 +4,8 @@ Tolerance (bf16 inputs, fp32 accumulation): max-abs <= 1e-2 and relative
 L2 <= 5e-3, on `out` and on `lse`.  Context rows beyond L_n are NaN on the
 device in every decode case, so any read of them would show.
 """
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -16,12 +18,33 @@ from two_tower_block_b200.workloads import WORKLOADS, make_causal, make_decode, 
 
 pytestmark = pytest.mark.gpu
 
-KERNELS = [pytest.param(ops.KERNEL_TCGEN05, id="tcgen05"), pytest.param(ops.KERNEL_MMA_SYNC, id="mma_sync")]
+# (kernel, tcgen05 key tile): the tcgen05 kernel runs with one 128-key S buffer per
+# M-tile (default) or two 64-key buffers (TT_TCGEN05_KEY_TILE=64, read at plan time)
+KERNELS = [pytest.param((ops.KERNEL_TCGEN05, None), id="tcgen05"),
+           pytest.param((ops.KERNEL_TCGEN05, "64"), id="tcgen05_k64"),
+           pytest.param((ops.KERNEL_MMA_SYNC, None), id="mma_sync")]
+
+
+def make_plan(kernel, *args, **kw):
+    """ops.Plan for a (kernel, key tile) parameter."""
+    kind, key_tile = kernel
+    old = os.environ.pop("TT_TCGEN05_KEY_TILE", None)
+    try:
+        if key_tile:
+            os.environ["TT_TCGEN05_KEY_TILE"] = key_tile
+        plan = ops.Plan(*args, kernel=kind, **kw)
+    finally:
+        os.environ.pop("TT_TCGEN05_KEY_TILE", None)
+        if old is not None:
+            os.environ["TT_TCGEN05_KEY_TILE"] = old
+    if key_tile:
+        assert plan.info().key_tile == int(key_tile)
+    return plan
 
 
 def run_decode(inp, kernel, num_ctas=0, poison=True):
     B, S, Hq, Hkv, D, Lcap = inp.shape
-    plan = ops.Plan(B, Hq, Hkv, D, S, ctx_capacity=Lcap, kernel=kernel, num_ctas=num_ctas)
+    plan = make_plan(kernel, B, Hq, Hkv, D, S, ctx_capacity=Lcap, num_ctas=num_ctas)
     kc = poison_beyond(inp.k_ctx, inp.ctx_lens) if poison else inp.k_ctx
     vc = poison_beyond(inp.v_ctx, inp.ctx_lens) if poison else inp.v_ctx
     out, lse = plan.block_attn(dev(inp.q), dev(kc), dev(vc), dev(inp.k_blk), dev(inp.v_blk),
@@ -112,7 +135,7 @@ def test_decode_long_L131072_sampled(kernel):
 def run_causal(inp, kernel, num_ctas=0):
     B, N, Hq, D = inp.q.shape
     Hkv = inp.k_ctx.shape[1]
-    plan = ops.Plan(B, Hq, Hkv, D, inp.block_size, seq_len=N, kernel=kernel, num_ctas=num_ctas)
+    plan = make_plan(kernel, B, Hq, Hkv, D, inp.block_size, seq_len=N, num_ctas=num_ctas)
     out, lse = plan.block_attn_block_causal(dev(inp.q), dev(inp.k_ctx), dev(inp.v_ctx), dev(inp.k_blk),
                                             dev(inp.v_blk), want_lse=True)
     plan.check()
@@ -158,7 +181,7 @@ def test_block_causal_equals_decode(kernel):
     out_c, lse_c = run_causal(inp, kernel)
     for b in [0, 1, 5]:
         p = slice(S * b, S * b + S)
-        plan = ops.Plan(B, Hq, Hkv, D, S, ctx_capacity=N, kernel=kernel)
+        plan = make_plan(kernel, B, Hq, Hkv, D, S, ctx_capacity=N)
         lens = torch.full((B,), S * b, dtype=torch.int32, device="cuda")
         out_d, lse_d = plan.block_attn(dev(np.ascontiguousarray(inp.q[:, p])), dev(inp.k_ctx), dev(inp.v_ctx),
                                        dev(np.ascontiguousarray(inp.k_blk[:, p])),
@@ -173,7 +196,7 @@ def test_host_io_entry_matches_device_entry(kernel):
     inp = make_decode(2, 16, 32, 2, 128, 600, seed=51, ctx_lens=[600, 257])
     B, S, Hq, Hkv, D, Lcap = inp.shape
     out_dev, lse_dev = run_decode(inp, kernel, poison=False)
-    plan = ops.Plan(B, Hq, Hkv, D, S, ctx_capacity=Lcap, kernel=kernel, host_io=True)
+    plan = make_plan(kernel, B, Hq, Hkv, D, S, ctx_capacity=Lcap, host_io=True)
 
     def pinned(bits):
         return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).pin_memory()
@@ -190,7 +213,7 @@ def test_host_io_entry_matches_device_entry(kernel):
 def test_ctx_len_out_of_range_is_reported(kernel):
     inp = make_decode(2, 16, 8, 2, 64, 100, seed=61, ctx_lens=[100, 50])
     B, S, Hq, Hkv, D, Lcap = inp.shape
-    plan = ops.Plan(B, Hq, Hkv, D, S, ctx_capacity=Lcap, kernel=kernel)
+    plan = make_plan(kernel, B, Hq, Hkv, D, S, ctx_capacity=Lcap)
     args = [dev(inp.q), dev(inp.k_ctx), dev(inp.v_ctx), dev(inp.k_blk), dev(inp.v_blk)]
     bad = torch.tensor([101, 50], dtype=torch.int32, device="cuda")
     plan.block_attn(*args, bad)
@@ -215,7 +238,7 @@ def test_wait_timeout_selftest():
 
 @pytest.mark.parametrize("kernel", KERNELS)
 def test_empty_batch_is_noop(kernel):
-    plan = ops.Plan(0, 8, 2, 128, 16, ctx_capacity=64, kernel=kernel)
+    plan = make_plan(kernel, 0, 8, 2, 128, 16, ctx_capacity=64)
     e = torch.empty(0, dtype=torch.bfloat16, device="cuda")
     lens = torch.empty(0, dtype=torch.int32, device="cuda")
     out = torch.empty(0, dtype=torch.float32, device="cuda")
@@ -227,7 +250,7 @@ def test_empty_batch_is_noop(kernel):
 def test_profile_hook_counts_launches(kernel):
     inp = make_decode(2, 16, 32, 2, 128, 2048, seed=71)
     B, S, Hq, Hkv, D, Lcap = inp.shape
-    plan = ops.Plan(B, Hq, Hkv, D, S, ctx_capacity=Lcap, kernel=kernel)
+    plan = make_plan(kernel, B, Hq, Hkv, D, S, ctx_capacity=Lcap)
     args = [dev(inp.q), dev(inp.k_ctx), dev(inp.v_ctx), dev(inp.k_blk), dev(inp.v_blk),
             torch.from_numpy(inp.ctx_lens).cuda()]
     plan.profile(True)

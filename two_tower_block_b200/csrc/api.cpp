@@ -6,6 +6,7 @@
 #include <algorithm>
 #include <cmath>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <string>
@@ -261,10 +262,15 @@ tt_status_t tt_block_attn_plan(const tt_block_attn_desc* desc, int device, tt_pl
   P->kernel = d.kernel == TT_KERNEL_AUTO ? TT_KERNEL_TCGEN05 : d.kernel;
   if (P->kernel == TT_KERNEL_TCGEN05 && prop.major != 10) P->kernel = TT_KERNEL_MMA_SYNC;
   if (P->kernel == TT_KERNEL_TCGEN05) {
-    P->key_tile = 128;
+    P->key_tile = tt::kTcgen05KeyTile;
+    // tuning knob: TT_TCGEN05_KEY_TILE=64 selects the two-buffer 64-key pipeline
+    if (const char* kt = std::getenv("TT_TCGEN05_KEY_TILE")) {
+      const int v = std::atoi(kt);
+      if (tt::tcgen05_key_tile_supported(v)) P->key_tile = v;
+    }
     P->C = d.num_ctas > 0 ? d.num_ctas : P->sm_count;
   } else {
-    P->key_tile = 64;
+    P->key_tile = tt::kMmaSyncKeyTile;
     const int rb = (P->R + 63) / 64;
     P->C = d.num_ctas > 0 ? d.num_ctas : std::max(1, (4 * P->sm_count) / rb);
   }

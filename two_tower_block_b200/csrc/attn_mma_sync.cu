@@ -15,7 +15,7 @@ namespace tt {
 namespace {
 
 constexpr int kRows = 64;   // packed query rows per CTA
-constexpr int kKeys = 64;   // keys per tile
+constexpr int kKeys = kMmaSyncKeyTile;  // keys per tile
 constexpr int kThreads = 128;
 
 template <int D>
@@ -157,10 +157,11 @@ __global__ void __launch_bounds__(kThreads) attn_mma_sync_kernel(const Problem p
       float rs0 = 0.f, rs1 = 0.f;
 #pragma unroll
       for (int nb = 0; nb < kKeys / 8; ++nb) {
-        s[nb][0] = fast_exp2(s[nb][0] - mn0);
-        s[nb][1] = fast_exp2(s[nb][1] - mn0);
-        s[nb][2] = fast_exp2(s[nb][2] - mn1);
-        s[nb][3] = fast_exp2(s[nb][3] - mn1);
+        // weights rounded to bf16 here, so the row sum uses what the PV product uses
+        s[nb][0] = __bfloat162float(__float2bfloat16_rn(fast_exp2(s[nb][0] - mn0)));
+        s[nb][1] = __bfloat162float(__float2bfloat16_rn(fast_exp2(s[nb][1] - mn0)));
+        s[nb][2] = __bfloat162float(__float2bfloat16_rn(fast_exp2(s[nb][2] - mn1)));
+        s[nb][3] = __bfloat162float(__float2bfloat16_rn(fast_exp2(s[nb][3] - mn1)));
         rs0 += s[nb][0] + s[nb][1];
         rs1 += s[nb][2] + s[nb][3];
       }

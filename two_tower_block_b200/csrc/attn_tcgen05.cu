@@ -15,16 +15,22 @@
 //                key tile into a ring of shared-memory slots (128-byte swizzle);
 //                for a tile whose valid rows are not a multiple of 16 it zeroes
 //                the V rows the last MMA k-step would otherwise read.
-//   warp 1       TMEM owner and MMA issuer (one thread): S_m = Q_m K^T into
-//                TMEM, O_m += P_m V with P read from TMEM (aliasing S_m).
+//   warp 1       TMEM owner and MMA issuer (one thread): S = Q_m K^T into TMEM,
+//                O_m += P V with P read from TMEM (aliasing its S buffer).
 //   warps 4..7   softmax warpgroup of M-tile 0 (thread = TMEM lane = row)
 //   warps 8..11  softmax warpgroup of M-tile 1
-// TMEM columns: S_0 [0,128), S_1 [128,256), O_0 [256,256+D), O_1 [256+D, 256+2D).
+// TMEM columns: M-tile m owns S buffers [128m, 128m+128) (NBUF buffers of NK
+// keys), O_0 = [256, 256+D), O_1 = [256+D, 256+2D).
+//
+// Pipeline per M-tile (tile G of the CTA uses S buffer G % NBUF): the MMA
+// thread issues PV(j) as soon as P(j) is ready and then S(j+NBUF) into the
+// buffer PV(j) has just consumed; with two buffers the softmax of tile j+1
+// finds its S ready while the tensor core works on PV(j).
 //
 // The softmax keeps a running reference maximum per row and rescales O (in
 // TMEM) only when a new maximum exceeds it by more than 2^8; the final
-// normalisation divides by the sum taken against the same reference, so the
-// result is exact up to rounding.
+// normalisation divides by the sum of the same bf16-rounded weights the PV
+// product used, so the result is exact up to rounding.
 //
 // Every wait is bounded (ptx.cuh: mbar_wait); on a timeout the CTA raises the
 // error word, drains what it issued, frees TMEM and returns.
@@ -36,33 +42,35 @@ namespace tt {
 namespace {
 
 constexpr int kThreads = 384;
-constexpr int kKeyTile = 128;
 constexpr int kMaxRows = 256;
 constexpr int kRowBytes = 128;              // one 64-element bf16 row of a swizzled half
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
-// Register split per warpgroup (launch: 168 per thread = 65536 / 384 rounded down to 8):
-// control warpgroup (warps 0-3) 4 x 32 x kCtrlRegs + softmax (warps 4-11) 8 x 32 x kSoftmaxRegs.
-constexpr int kCtrlRegs = 80;
-constexpr int kSoftmaxRegs = 200;
-static_assert(4 * 32 * kCtrlRegs + 8 * 32 * kSoftmaxRegs <= kThreads * 168, "register split exceeds the launch");
 
-template <int D>
+template <int D, int NK>
 struct Cfg {
   static constexpr int kHalves = D / 64;
-  static constexpr int kStages = D == 128 ? 4 : 8;
+  static constexpr int kBufs = 128 / NK;                       // S buffers per M-tile
+  static constexpr int kSlotBytes = NK * kRowBytes * kHalves;  // one K or V tile
+  static constexpr int kStages = (128 * 1024) / kSlotBytes;    // 128 KB ring
   static constexpr int kQBytes = kMaxRows * kRowBytes * kHalves;
-  static constexpr int kSlotBytes = kKeyTile * kRowBytes * kHalves;
   static constexpr int kStageOff = kQBytes;
   static constexpr int kEpiOff = kStageOff + kStages * kSlotBytes;
   static constexpr int kEpiBytes = 8 * 32 * 32 * 4;  // 8 softmax warps x 32 rows x 32 fp32
   static constexpr int kBarOff = kEpiOff + kEpiBytes;
   static constexpr int kSmemBytes = kBarOff + 512 + 1024;  // barriers/flags + alignment slack
+  // Register split (launch: 168 per thread = 65536 / 384 rounded down to 8): the
+  // 128-key variant keeps a full 128-score row per softmax thread.
+  static constexpr bool kSplitRegs = NK == 128;
+  static constexpr int kCtrlRegs = 80, kSoftmaxRegs = 200;
+  static_assert(4 * 32 * kCtrlRegs + 8 * 32 * kSoftmaxRegs <= kThreads * 168, "register split");
+  static_assert(kStages <= 16, "ring too deep");
 };
 
 struct Bars {
   uint64_t q_full, q_empty, tail, drain;
-  uint64_t s_full[2], p_full[2], o_full[2], o_empty[2];
-  uint64_t kv_full[8], kv_empty[8];
+  uint64_t s_full[2][2], p_full[2][2];  // [M-tile][S buffer]
+  uint64_t pv_done[2], o_full[2], o_empty[2];
+  uint64_t kv_full[16], kv_empty[16];
 };
 
 struct Shared {
@@ -83,29 +91,30 @@ __device__ __forceinline__ float* out_row(const Problem& p, const Unit& x, const
   return p.part_o + ((size_t)sg.slot * p.R + r) * D;
 }
 
-// Row maximum of the first `count` raw scores of a tile (all kKeyTile when kFull).
-template <bool kFull>
+// Row maximum of the first `count` raw scores of a tile (all NK when kFull).
+template <int NK, bool kFull>
 __device__ __forceinline__ float tile_row_max(const uint32_t* v, int count) {
   float m[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-  for (int k = 0; k < kKeyTile; ++k) {
+  for (int k = 0; k < NK; ++k) {
     const float x = __uint_as_float(v[k]);
     m[k & 3] = fmaxf(m[k & 3], (kFull || k < count) ? x : -INFINITY);
   }
   return fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
 }
 
-// p = 2^(s*c - m_ref) for the tile's keys (0 beyond `count`), written to TMEM as bf16
-// pairs over the first columns of the S region: keys [32ch, 32ch+32) -> columns
-// [16ch, 16ch+16).  Returns the row sum of p (fp32, before the bf16 rounding).
-template <bool kFull>
+// p = 2^(s*c - m_ref) for the tile's keys (0 beyond `count`), rounded to bf16 and
+// written to TMEM as pairs over the first columns of the S buffer: keys
+// [32ch, 32ch+32) -> columns [16ch, 16ch+16).  Returns the row sum of the
+// rounded weights, so that numerator and denominator use the same values.
+template <int NK, bool kFull>
 __device__ __forceinline__ float tile_exp_store(const uint32_t* v, int count, float c, float m_ref,
                                                 uint32_t s_addr) {
   const float2 c2 = make_float2(c, c);
   const float2 nm2 = make_float2(-m_ref, -m_ref);
   float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
-  for (int ch = 0; ch < kKeyTile / 32; ++ch) {
+  for (int ch = 0; ch < NK / 32; ++ch) {
     if (!kFull && 32 * ch >= count) break;
     uint32_t pk[16];
 #pragma unroll
@@ -117,18 +126,20 @@ __device__ __forceinline__ float tile_exp_store(const uint32_t* v, int count, fl
         a = c0 < count ? a : 0.f;
         b = c0 + 1 < count ? b : 0.f;
       }
-      acc = __fadd2_rn(acc, make_float2(a, b));
-      pk[k] = pack_bf16(a, b);
+      const uint32_t h = pack_bf16(a, b);
+      pk[k] = h;
+      acc = __fadd2_rn(acc, make_float2(__uint_as_float(h << 16), __uint_as_float(h & 0xFFFF0000u)));
     }
     tmem_st16(s_addr + 16 * ch, pk);
   }
   return acc.x + acc.y;
 }
 
-template <int D>
+template <int D, int NK>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tcgen05_kernel(const Problem p, const __grid_constant__ TmaMaps maps) {
-  using C = Cfg<D>;
+  using C = Cfg<D, NK>;
+  constexpr int NBUF = C::kBufs;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   const uint32_t sbase = smem_u32(smem);
@@ -155,8 +166,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(smem_u32(&bars->tail), 1);
     mbar_init(smem_u32(&bars->drain), 1);
     for (int m = 0; m < 2; ++m) {
-      mbar_init(smem_u32(&bars->s_full[m]), 1);
-      mbar_init(smem_u32(&bars->p_full[m]), 128);
+      for (int b = 0; b < 2; ++b) {
+        mbar_init(smem_u32(&bars->s_full[m][b]), 1);
+        mbar_init(smem_u32(&bars->p_full[m][b]), 128);
+      }
+      mbar_init(smem_u32(&bars->pv_done[m]), 1);
       mbar_init(smem_u32(&bars->o_full[m]), 1);
       mbar_init(smem_u32(&bars->o_empty[m]), 128);
     }
@@ -197,8 +211,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const long long T = sh->T, start = sh->start, end = sh->end;
   const WaitCtx wc{&sh->abort_flag, p.err_word, p.wait_limit_ns};
   const bool have_work = start < end;
+  if constexpr (C::kSplitRegs) {
+    if (have_work && warp < 4) regs_dec<C::kCtrlRegs>();
+  }
 
-  if (have_work && warp < 4) regs_dec<kCtrlRegs>();
   if (warp == 0 && have_work) {
     // ============================================================ producer ==
     uint32_t it = 0, q_it = 0, tail_ph = 0;
@@ -218,7 +234,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int ctx_row0 = (x.n * p.Hkv + x.h) * p.ctx_stride;
       for (int i = sg.lo; i < sg.hi && ok; ++i) {
         const TileKeys tk = tile_keys(p, x, i);
-        const int box_rows = tk.is_blk ? min(p.S, kKeyTile) : kKeyTile;
+        const int box_rows = tk.is_blk ? min(p.S, NK) : NK;
         const uint32_t bytes = (uint32_t)(box_rows * kRowBytes * C::kHalves);
         for (int kv = 0; kv < 2 && ok; ++kv, ++it) {
           const int s = it % C::kStages;
@@ -232,7 +248,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (lane == 0) {
             mbar_arrive_expect_tx(bar, bytes);
             for (int hf = 0; hf < C::kHalves; ++hf) {
-              const uint32_t dst = slot + hf * (kKeyTile * kRowBytes);
+              const uint32_t dst = slot + hf * (NK * kRowBytes);
               if (tk.is_blk) tma_load_3d(dst, m, bar, hf * 64, x.h, x.ns * p.S + tk.first);
               else tma_load_2d(dst, m, bar, hf * 64, ctx_row0 + tk.first);
             }
@@ -248,7 +264,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               const int rem = e - hf * (r1 - r0) * 8;
               const int row = r0 + rem / 8, ch = rem % 8;
               uint4* dst = reinterpret_cast<uint4*>(smem + C::kStageOff + s * C::kSlotBytes +
-                                                    hf * (kKeyTile * kRowBytes) + row * kRowBytes + ch * 16);
+                                                    hf * (NK * kRowBytes) + row * kRowBytes + ch * 16);
               *dst = make_uint4(0, 0, 0, 0);
             }
             fence_proxy_async_smem();
@@ -262,9 +278,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (!ok) {
       // drain: wait (briefly) for loads that may still be landing in shared memory
-      WaitCtx dw{&sh->abort_flag, nullptr, 2000000ull};
       int dummy = 0;
-      dw.abort_flag = &dummy;
+      WaitCtx dw{&dummy, nullptr, 2000000ull};
       for (uint32_t j = (it > (uint32_t)C::kStages ? it - C::kStages : 0); j < it; ++j)
         mbar_wait(smem_u32(&bars->kv_full[j % C::kStages]), (j / C::kStages) & 1, dw);
       if (q_it) mbar_wait(smem_u32(&bars->q_full), (q_it - 1) & 1, dw);
@@ -272,74 +287,85 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1 && have_work) {
     // ============================================================= MMA warp ==
     if (lane == 0) {
-      uint32_t it = 0, q_it = 0, t_cnt = 0, seg_cnt = 0;
+      uint32_t it = 0, q_it = 0, G = 0, seg_cnt = 0;
       bool ok = true;
       Unit x = sh->first;
+      // descriptors: a start-address offset is added in 16-byte units to the low field
+      const uint64_t qdesc = smem_desc_sw128(q_s, 16, 1024);
+      const uint64_t kdesc0 = smem_desc_sw128(kv_s, 16, 1024);
+      const uint64_t vdesc0 = smem_desc_sw128(kv_s, NK * kRowBytes, 1024);
       const uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
+      const uint32_t idesc_s0 = idesc_bf16_f32(128, 0, 0, 0);
+      auto issue_s = [&](int m, int buf, uint32_t slot, int n_mma) {
+        const uint32_t idesc = idesc_s0 | ((uint32_t)(n_mma >> 3) << 17);
+        const uint64_t kd = kdesc0 + (uint64_t)((slot * C::kSlotBytes) >> 4);
+        const uint64_t qd = qdesc + (uint64_t)((m * 128 * kRowBytes) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * (kMaxRows * kRowBytes) + (kk & 3) * 32;
+          const uint32_t koff = (kk >> 2) * (NK * kRowBytes) + (kk & 3) * 32;
+          tc_mma_ss(tmem + m * 128 + buf * NK, qd + (off >> 4), kd + (koff >> 4), idesc, kk > 0);
+        }
+      };
+      auto kv_wait = [&](uint32_t e) {
+        return mbar_wait(smem_u32(&bars->kv_full[e % C::kStages]), (e / C::kStages) & 1, wc);
+      };
       for (; ok;) {
         const Segment sg = segment_of(x, start, end, c);
+        const int n = sg.hi - sg.lo;
         ok = mbar_wait(smem_u32(&bars->q_full), q_it & 1, wc);
         ++q_it;
         if (!ok) break;
         tc_fence_after();
-        // S_m(i) = Q_m K_i^T
-        auto issue_s = [&](int m, uint32_t kslot, int n_mma) {
-          const uint32_t idesc = idesc_bf16_f32(128, n_mma, 0, 0);
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const int hf = kk >> 2, ko = (kk & 3) * 32;
-            const uint64_t a = smem_desc_sw128(q_s + hf * (kMaxRows * kRowBytes) + m * 128 * kRowBytes + ko, 16, 1024);
-            const uint64_t b = smem_desc_sw128(kslot + hf * (kKeyTile * kRowBytes) + ko, 16, 1024);
-            tc_mma_ss(tmem + m * 128, a, b, idesc, kk > 0);
-          }
-        };
-        // prologue: S of the first tile
-        {
-          const int n0 = round16(tile_keys(p, x, sg.lo).count);
-          const int s = it % C::kStages;
-          ok = mbar_wait(smem_u32(&bars->kv_full[s]), (it / C::kStages) & 1, wc);
+        // prologue: S of the segment's first NBUF tiles (K of tile j = ring entry it + 2j)
+        for (int j = 0; j < NBUF && j < n && ok; ++j) {
+          ok = kv_wait(it + 2 * j);
           if (!ok) break;
           tc_fence_after();
+          const int nk = round16(tile_keys(p, x, sg.lo + j).count);
+          const uint32_t ks = (it + 2 * j) % C::kStages;
           for (int m = 0; m < MT; ++m) {
-            issue_s(m, kv_s + s * C::kSlotBytes, n0);
-            tc_commit(smem_u32(&bars->s_full[m]));
+            issue_s(m, (G + j) % NBUF, ks, nk);
+            tc_commit(smem_u32(&bars->s_full[m][(G + j) % NBUF]));
           }
-          tc_commit(smem_u32(&bars->kv_empty[s]));
+          tc_commit(smem_u32(&bars->kv_empty[ks]));
         }
-        for (int i = sg.lo; i < sg.hi && ok; ++i, ++t_cnt) {
-          const int nv = round16(tile_keys(p, x, i).count);
-          const int sv = (it + 1) % C::kStages;
-          ok = mbar_wait(smem_u32(&bars->kv_full[sv]), ((it + 1) / C::kStages) & 1, wc);
+        for (int j = 0; j < n && ok; ++j, ++G) {
+          const int b = G % NBUF;
+          const uint32_t ev = it + 2 * j + 1;  // V of tile j
+          ok = kv_wait(ev);
           if (!ok) break;
-          const bool more = i + 1 < sg.hi;
-          const int sk2 = (it + 2) % C::kStages;
-          const int nn = more ? round16(tile_keys(p, x, i + 1).count) : 0;
+          const int nv = round16(tile_keys(p, x, sg.lo + j).count);
+          const bool ahead = j + NBUF < n;     // S of tile j + NBUF goes into buffer b
+          const uint32_t ek = it + 2 * (j + NBUF);
+          const int nk = ahead ? round16(tile_keys(p, x, sg.lo + j + NBUF).count) : 0;
+          const uint64_t vd = vdesc0 + (uint64_t)(((ev % C::kStages) * C::kSlotBytes) >> 4);
           for (int m = 0; m < MT && ok; ++m) {
-            ok = mbar_wait(smem_u32(&bars->p_full[m]), t_cnt & 1, wc);
-            if (ok && i == sg.lo) ok = mbar_wait(smem_u32(&bars->o_empty[m]), (seg_cnt & 1) ^ 1, wc);
+            ok = mbar_wait(smem_u32(&bars->p_full[m][b]), (G / NBUF) & 1, wc);
+            if (ok && j == 0) ok = mbar_wait(smem_u32(&bars->o_empty[m]), (seg_cnt & 1) ^ 1, wc);
             if (!ok) break;
             tc_fence_after();
-            const uint32_t vslot = kv_s + sv * C::kSlotBytes;
-            for (int kk = 0; kk < nv / 16; ++kk) {
-              const uint64_t b = smem_desc_sw128(vslot + kk * 16 * kRowBytes, kKeyTile * kRowBytes, 1024);
-              tc_mma_ts(tmem + 256 + m * D, tmem + m * 128 + kk * 8, b, idesc_pv, (i > sg.lo || kk > 0) ? 1u : 0u);
-            }
-            if (more) {
+            const uint32_t pa = tmem + m * 128 + b * NK;
+            for (int kk = 0; kk < nv / 16; ++kk)
+              tc_mma_ts(tmem + 256 + m * D, pa + kk * 8, vd + (uint64_t)(kk * 16 * kRowBytes >> 4), idesc_pv,
+                        (j > 0 || kk > 0) ? 1u : 0u);
+            tc_commit(smem_u32(&bars->pv_done[m]));
+            if (ahead) {
               if (m == 0) {
-                ok = mbar_wait(smem_u32(&bars->kv_full[sk2]), ((it + 2) / C::kStages) & 1, wc);
+                ok = kv_wait(ek);
                 if (!ok) break;
                 tc_fence_after();
               }
-              issue_s(m, kv_s + sk2 * C::kSlotBytes, nn);
-              tc_commit(smem_u32(&bars->s_full[m]));
+              issue_s(m, b, ek % C::kStages, nk);
+              tc_commit(smem_u32(&bars->s_full[m][b]));
             }
           }
           if (!ok) break;
-          tc_commit(smem_u32(&bars->kv_empty[sv]));
-          if (more) tc_commit(smem_u32(&bars->kv_empty[sk2]));
-          it += 2;
+          tc_commit(smem_u32(&bars->kv_empty[ev % C::kStages]));
+          if (ahead) tc_commit(smem_u32(&bars->kv_empty[ek % C::kStages]));
         }
         if (!ok) break;
+        it += 2 * n;
         for (int m = 0; m < MT; ++m) tc_commit(smem_u32(&bars->o_full[m]));
         tc_commit(smem_u32(&bars->q_empty));
         ++seg_cnt;
@@ -355,40 +381,46 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp >= 4 && have_work) {
     // ========================================================= softmax WGs ==
-    regs_inc<kSoftmaxRegs>();
+    if constexpr (C::kSplitRegs) regs_inc<C::kSoftmaxRegs>();
     const int m = (warp - 4) >> 2;
     const int q4 = warp & 3;             // TMEM lane quarter of this warp
     const int row = q4 * 32 + lane;      // row within the M-tile
     const int r = m * 128 + row;         // packed row of the unit
     if (m < MT) {
       const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
-      const uint32_t s_addr = tmem + lane_off + m * 128;
+      const uint32_t s_base = tmem + lane_off + m * 128;  // + buffer * NK
       const uint32_t o_addr = tmem + lane_off + 256 + m * D;
       float* stage = epi + (warp - 4) * 32 * 32;
-      uint32_t t_cnt = 0, seg_cnt = 0;
+      uint32_t G = 0, seg_cnt = 0;
       bool ok = true;
       Unit x = sh->first;
       for (; ok;) {
         const Segment sg = segment_of(x, start, end, c);
         float m_ref = -INFINITY, l = 0.f;
-        for (int i = sg.lo; i < sg.hi; ++i, ++t_cnt) {
+        for (int i = sg.lo; i < sg.hi; ++i, ++G) {
           const int count = tile_keys(p, x, i).count;
-          ok = mbar_wait(smem_u32(&bars->s_full[m]), t_cnt & 1, wc);
+          const int b = G % NBUF;
+          const uint32_t s_addr = s_base + b * NK;
+          ok = mbar_wait(smem_u32(&bars->s_full[m][b]), (G / NBUF) & 1, wc);
           if (!ok) break;
           tc_fence_after();
           // the tile's S row in registers; row maximum in log2 units (masked beyond `count`)
-          const bool full = count == kKeyTile;
-          uint32_t v[kKeyTile];
+          const bool full = count == NK;
+          uint32_t v[NK];
 #pragma unroll
-          for (int ch = 0; ch < kKeyTile / 32; ++ch)
+          for (int ch = 0; ch < NK / 32; ++ch)
             if (full || 32 * ch < count) tmem_ld32(s_addr + 32 * ch, v + 32 * ch);
           tc_wait_ld();
-          const float mx = (full ? tile_row_max<true>(v, count) : tile_row_max<false>(v, count)) * p.scale_log2;
+          const float mx = (full ? tile_row_max<NK, true>(v, count) : tile_row_max<NK, false>(v, count)) * p.scale_log2;
           if (i == sg.lo) {
             m_ref = mx;  // O is overwritten by the first PV of the segment
           } else {
             const bool need = mx > m_ref + kRescaleThreshold;
             if (__any_sync(0xffffffffu, need)) {
+              // O must hold every earlier PV of this segment before it is rescaled
+              ok = mbar_wait(smem_u32(&bars->pv_done[m]), (G - 1) & 1, wc);
+              if (!ok) break;
+              tc_fence_after();
               const float alpha = need ? fast_exp2(m_ref - mx) : 1.f;
               if (need) {
                 m_ref = mx;
@@ -405,13 +437,11 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
             }
           }
-          const float sum = full ? tile_exp_store<true>(v, count, p.scale_log2, m_ref, s_addr)
-                                 : tile_exp_store<false>(v, count, p.scale_log2, m_ref, s_addr);
-          l += sum;
-          if (!ok) break;
+          l += full ? tile_exp_store<NK, true>(v, count, p.scale_log2, m_ref, s_addr)
+                    : tile_exp_store<NK, false>(v, count, p.scale_log2, m_ref, s_addr);
           tc_wait_st();
           tc_fence_before();
-          mbar_arrive(smem_u32(&bars->p_full[m]));
+          mbar_arrive(smem_u32(&bars->p_full[m][b]));
         }
         if (!ok) break;
         // ---- epilogue: O / l to the output (or the segment's partial) ----
@@ -484,25 +514,38 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
+template <int D, int NK>
+void set_smem_attr() {
+  cudaFuncSetAttribute(attn_tcgen05_kernel<D, NK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       Cfg<D, NK>::kSmemBytes);
+}
+
+template <int D, int NK>
+void launch(const Problem& p, const TmaMaps& maps, cudaStream_t stream) {
+  attn_tcgen05_kernel<D, NK><<<p.C, kThreads, Cfg<D, NK>::kSmemBytes, stream>>>(p, maps);
+}
+
 }  // namespace
 
-size_t attn_tcgen05_smem_bytes(int D) {
-  return D == 128 ? (size_t)Cfg<128>::kSmemBytes : (size_t)Cfg<64>::kSmemBytes;
-}
+bool tcgen05_key_tile_supported(int key_tile) { return key_tile == 64 || key_tile == 128; }
 
 cudaError_t launch_attn_tcgen05(const Problem& p, const TmaMaps& maps, cudaStream_t stream) {
   static const bool attr_done = [] {
-    cudaFuncSetAttribute(attn_tcgen05_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         Cfg<128>::kSmemBytes);
-    cudaFuncSetAttribute(attn_tcgen05_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         Cfg<64>::kSmemBytes);
+    set_smem_attr<128, 128>();
+    set_smem_attr<128, 64>();
+    set_smem_attr<64, 128>();
+    set_smem_attr<64, 64>();
     return true;
   }();
   (void)attr_done;
-  if (p.D == 128)
-    attn_tcgen05_kernel<128><<<p.C, kThreads, Cfg<128>::kSmemBytes, stream>>>(p, maps);
-  else
-    attn_tcgen05_kernel<64><<<p.C, kThreads, Cfg<64>::kSmemBytes, stream>>>(p, maps);
+  if (!tcgen05_key_tile_supported(p.key_tile)) return cudaErrorInvalidValue;
+  if (p.D == 128) {
+    if (p.key_tile == 128) launch<128, 128>(p, maps, stream);
+    else launch<128, 64>(p, maps, stream);
+  } else {
+    if (p.key_tile == 128) launch<64, 128>(p, maps, stream);
+    else launch<64, 64>(p, maps, stream);
+  }
   return cudaGetLastError();
 }
 

@@ -136,7 +136,7 @@ extern "C" TT_API tt_status_t tt_block_attn_noalloc(const tt_block_attn_desc* de
   if (st != TT_OK) return st;
 
   const int kernel = (d.kernel == TT_KERNEL_MMA_SYNC || ds->major != 10) ? TT_KERNEL_MMA_SYNC : TT_KERNEL_TCGEN05;
-  const int key_tile = kernel == TT_KERNEL_TCGEN05 ? 128 : 64;
+  const int key_tile = kernel == TT_KERNEL_TCGEN05 ? tt::kTcgen05KeyTile : tt::kMmaSyncKeyTile;
   int C = d.num_ctas;
   if (C == 0) {
     C = kernel == TT_KERNEL_TCGEN05 ? ds->sm_count : std::max(1, (4 * ds->sm_count) / ((R + 63) / 64));

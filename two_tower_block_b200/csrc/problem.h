@@ -11,6 +11,12 @@ namespace tt {
 
 enum Mode : int { kDecode = 0, kBlockCausal = 1 };
 
+// Keys per pipeline tile of each kernel (the work split counts tiles of this size).
+// The tcgen05 kernel also runs with 64-key tiles and two S buffers per M-tile
+// (see tcgen05_key_tile_supported); 128 is the default.
+constexpr int kTcgen05KeyTile = 128;
+constexpr int kMmaSyncKeyTile = 64;
+
 struct Problem {
   // geometry
   int mode;        // kDecode or kBlockCausal
@@ -50,6 +56,7 @@ struct TmaMaps {
   CUtensorMap q, k_ctx, v_ctx, k_blk, v_blk;
 };
 cudaError_t launch_attn_tcgen05(const Problem& p, const TmaMaps& maps, cudaStream_t stream);
+bool tcgen05_key_tile_supported(int key_tile);
 size_t attn_tcgen05_smem_bytes(int D);
 size_t attn_mma_sync_smem_bytes(int D);
 
