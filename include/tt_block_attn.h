@@ -193,6 +193,13 @@ TT_API tt_status_t tt_block_attn_profile_read(tt_plan_t plan, int kernel_id, int
  * the device context still usable afterwards. */
 TT_API tt_status_t tt_selftest_wait_timeout(int device, int timeout_us, tt_stream_t stream);
 
+/* Numerics self test: evaluates on the device the FMA-pipe exp2 the softmax uses
+ * for a quarter of its weights (range reduction plus a fitted degree-3 polynomial,
+ * maximum relative error 7.5e-5 for arguments in [-125, 127]) on the n host values
+ * x and writes the n results to y (host).  Synchronous; allocates its own
+ * buffers. */
+TT_API tt_status_t tt_selftest_exp2(int device, const float* x, float* y, int n);
+
 /* Host-only view of the work split (no GPU needed): for `num_units` units with
  * tiles_per_unit[u] tiles each over `num_ctas` ranges, writes for every range c
  * its first global tile (range_start[c], num_ctas+1 entries) and, per unit, the

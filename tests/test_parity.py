@@ -18,27 +18,30 @@ from two_tower_block_b200.workloads import WORKLOADS, make_causal, make_decode, 
 
 pytestmark = pytest.mark.gpu
 
-# (kernel, tcgen05 key tile): the tcgen05 kernel runs with one 128-key S buffer per
-# M-tile (default) or two 64-key buffers (TT_TCGEN05_KEY_TILE=64, read at plan time)
-KERNELS = [pytest.param((ops.KERNEL_TCGEN05, None), id="tcgen05"),
-           pytest.param((ops.KERNEL_TCGEN05, "64"), id="tcgen05_k64"),
-           pytest.param((ops.KERNEL_MMA_SYNC, None), id="mma_sync")]
+# (kernel, plan-time tuning knobs): the tcgen05 kernel with one 128-key S buffer per
+# M-tile (default), with two 64-key buffers (TT_TCGEN05_KEY_TILE=64), and the
+# transposed-PV kernel for head_dim 128 (TT_TCGEN05_VARIANT=2); the mma.sync baseline
+KERNELS = [pytest.param((ops.KERNEL_TCGEN05, {}), id="tcgen05"),
+           pytest.param((ops.KERNEL_TCGEN05, {"TT_TCGEN05_KEY_TILE": "64"}), id="tcgen05_k64"),
+           pytest.param((ops.KERNEL_TCGEN05, {"TT_TCGEN05_VARIANT": "2"}), id="tcgen05_pt"),
+           pytest.param((ops.KERNEL_MMA_SYNC, {}), id="mma_sync")]
+KNOBS = ("TT_TCGEN05_KEY_TILE", "TT_TCGEN05_VARIANT")
 
 
 def make_plan(kernel, *args, **kw):
-    """ops.Plan for a (kernel, key tile) parameter."""
-    kind, key_tile = kernel
-    old = os.environ.pop("TT_TCGEN05_KEY_TILE", None)
+    """ops.Plan for a (kernel, knobs) parameter; the knobs are read at plan creation."""
+    kind, knobs = kernel
+    old = {k: os.environ.pop(k, None) for k in KNOBS}
     try:
-        if key_tile:
-            os.environ["TT_TCGEN05_KEY_TILE"] = key_tile
+        os.environ.update(knobs)
         plan = ops.Plan(*args, kernel=kind, **kw)
     finally:
-        os.environ.pop("TT_TCGEN05_KEY_TILE", None)
-        if old is not None:
-            os.environ["TT_TCGEN05_KEY_TILE"] = old
-    if key_tile:
-        assert plan.info().key_tile == int(key_tile)
+        for k in KNOBS:
+            os.environ.pop(k, None)
+            if old[k] is not None:
+                os.environ[k] = old[k]
+    if "TT_TCGEN05_KEY_TILE" in knobs:
+        assert plan.info().key_tile == int(knobs["TT_TCGEN05_KEY_TILE"])
     return plan
 
 

@@ -82,6 +82,7 @@ struct tt_plan_s {
   int kernel = TT_KERNEL_MMA_SYNC;
   int C = 1;
   int key_tile = 64;
+  int variant = 0;
   int R = 0, g = 1;
   float scale = 0.f;
   // scratch
@@ -151,6 +152,7 @@ tt::Problem base_problem(tt_plan_t plan) {
   p.records = plan->records;
   p.err_word = plan->err_word;
   p.wait_limit_ns = (unsigned long long)(d.wait_timeout_us > 0 ? d.wait_timeout_us : 1000000) * 1000ull;
+  p.variant = plan->variant;
   return p;
 }
 
@@ -263,11 +265,13 @@ tt_status_t tt_block_attn_plan(const tt_block_attn_desc* desc, int device, tt_pl
   if (P->kernel == TT_KERNEL_TCGEN05 && prop.major != 10) P->kernel = TT_KERNEL_MMA_SYNC;
   if (P->kernel == TT_KERNEL_TCGEN05) {
     P->key_tile = tt::kTcgen05KeyTile;
-    // tuning knob: TT_TCGEN05_KEY_TILE=64 selects the two-buffer 64-key pipeline
+    // tuning knobs: TT_TCGEN05_KEY_TILE=64 selects the two-buffer 64-key pipeline;
+    // TT_TCGEN05_VARIANT=2 selects the transposed-PV kernel for head_dim 128
     if (const char* kt = std::getenv("TT_TCGEN05_KEY_TILE")) {
       const int v = std::atoi(kt);
       if (tt::tcgen05_key_tile_supported(v)) P->key_tile = v;
     }
+    if (const char* kv = std::getenv("TT_TCGEN05_VARIANT")) P->variant = std::atoi(kv) == 2 ? 2 : 0;
     P->C = d.num_ctas > 0 ? d.num_ctas : P->sm_count;
   } else {
     P->key_tile = tt::kMmaSyncKeyTile;
@@ -467,6 +471,7 @@ tt_status_t tt_block_attn_check(tt_plan_t plan, tt_stream_t stream) {
   e = cudaMemcpy(&w, plan->err_word, sizeof(w), cudaMemcpyDeviceToHost);
   if (e == cudaSuccess) e = cudaMemset(plan->err_word, 0, sizeof(unsigned));
   if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
+  if (w & tt::kErrInternal) return fail(TT_ERR_CUDA, "a kernel found its launch unusable (internal error)");
   if (w & tt::kErrTimeout) return fail(TT_ERR_TIMEOUT, "an in-kernel wait timed out");
   if (w & tt::kErrDeviceArg) return fail(TT_ERR_DEVICE_ARG, "ctx_lens value outside [0, ctx_capacity]");
   return TT_OK;
@@ -523,6 +528,22 @@ tt_status_t tt_selftest_wait_timeout(int device, int timeout_us, tt_stream_t str
   if (e != cudaSuccess) return cuda_fail(e, "wait self test");
   if (h & 0x80000000u) return fail(TT_ERR_INVALID_ARG, "self test: a wait on a barrier nothing arrives at returned");
   if (h & tt::kErrTimeout) return TT_ERR_TIMEOUT;
+  return TT_OK;
+}
+
+tt_status_t tt_selftest_exp2(int device, const float* x, float* y, int n) {
+  if (n < 0 || (n > 0 && (!x || !y))) return fail(TT_ERR_INVALID_ARG, "bad arguments");
+  if (n == 0) return TT_OK;
+  DeviceGuard guard(device);
+  float* d = nullptr;
+  cudaError_t e = cudaMalloc(&d, sizeof(float) * 2 * (size_t)n);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc");
+  e = cudaMemcpy(d, x, sizeof(float) * n, cudaMemcpyHostToDevice);
+  if (e == cudaSuccess) e = tt::launch_exp2_selftest(d, d + n, n, 0);
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  if (e == cudaSuccess) e = cudaMemcpy(y, d + n, sizeof(float) * n, cudaMemcpyDeviceToHost);
+  cudaFree(d);
+  if (e != cudaSuccess) return cuda_fail(e, "exp2 self test");
   return TT_OK;
 }
 

@@ -36,6 +36,7 @@
 // error word, drains what it issued, frees TMEM and returns.
 #include "problem.h"
 #include "ptx.cuh"
+#include "tc_common.cuh"
 #include "walker.cuh"
 
 namespace tt {
@@ -79,61 +80,6 @@ struct Shared {
   long long T, start, end;
   Unit first;
 };
-
-__device__ __forceinline__ int round16(int x) { return (x + 15) & ~15; }
-
-// Output row pointer of packed row r of unit x (final output or segment partial).
-__device__ __forceinline__ float* out_row(const Problem& p, const Unit& x, const Segment& sg, int r, int D) {
-  if (sg.full) {
-    const int t = r / p.g, j = r - (r / p.g) * p.g;
-    return p.out + ((size_t)(x.ns * p.S + t) * p.Hq + x.h * p.g + j) * D;
-  }
-  return p.part_o + ((size_t)sg.slot * p.R + r) * D;
-}
-
-// Row maximum of the first `count` raw scores of a tile (all NK when kFull).
-template <int NK, bool kFull>
-__device__ __forceinline__ float tile_row_max(const uint32_t* v, int count) {
-  float m[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-  for (int k = 0; k < NK; ++k) {
-    const float x = __uint_as_float(v[k]);
-    m[k & 3] = fmaxf(m[k & 3], (kFull || k < count) ? x : -INFINITY);
-  }
-  return fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
-}
-
-// p = 2^(s*c - m_ref) for the tile's keys (0 beyond `count`), rounded to bf16 and
-// written to TMEM as pairs over the first columns of the S buffer: keys
-// [32ch, 32ch+32) -> columns [16ch, 16ch+16).  Returns the row sum of the
-// rounded weights, so that numerator and denominator use the same values.
-template <int NK, bool kFull>
-__device__ __forceinline__ float tile_exp_store(const uint32_t* v, int count, float c, float m_ref,
-                                                uint32_t s_addr) {
-  const float2 c2 = make_float2(c, c);
-  const float2 nm2 = make_float2(-m_ref, -m_ref);
-  float2 acc = make_float2(0.f, 0.f);
-#pragma unroll
-  for (int ch = 0; ch < NK / 32; ++ch) {
-    if (!kFull && 32 * ch >= count) break;
-    uint32_t pk[16];
-#pragma unroll
-    for (int k = 0; k < 16; ++k) {
-      const int c0 = 32 * ch + 2 * k;
-      const float2 x = __ffma2_rn(make_float2(__uint_as_float(v[c0]), __uint_as_float(v[c0 + 1])), c2, nm2);
-      float a = fast_exp2(x.x), b = fast_exp2(x.y);
-      if (!kFull) {
-        a = c0 < count ? a : 0.f;
-        b = c0 + 1 < count ? b : 0.f;
-      }
-      const uint32_t h = pack_bf16(a, b);
-      pk[k] = h;
-      acc = __fadd2_rn(acc, make_float2(__uint_as_float(h << 16), __uint_as_float(h & 0xFFFF0000u)));
-    }
-    tmem_st16(s_addr + 16 * ch, pk);
-  }
-  return acc.x + acc.y;
-}
 
 template <int D, int NK>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -539,6 +485,8 @@ cudaError_t launch_attn_tcgen05(const Problem& p, const TmaMaps& maps, cudaStrea
   }();
   (void)attr_done;
   if (!tcgen05_key_tile_supported(p.key_tile)) return cudaErrorInvalidValue;
+  // variant 2: head_dim 128 with 128-key tiles on the transposed-PV kernel (attn_tcgen05_pt.cu)
+  if (p.D == 128 && p.key_tile == 128 && p.variant == 2) return launch_attn_pt(p, maps, stream);
   if (p.D == 128) {
     if (p.key_tile == 128) launch<128, 128>(p, maps, stream);
     else launch<128, 64>(p, maps, stream);

@@ -103,7 +103,24 @@ __global__ void wait_selftest_kernel(unsigned* err_word, unsigned long long limi
   __syncthreads();
 }
 
+// The FMA-pipe exp2 of the softmax (ptx.cuh: exp2_poly2) on n arguments.
+__global__ void exp2_selftest_kernel(const float* x, float* y, int n) {
+  const int i = (blockIdx.x * blockDim.x + threadIdx.x) * 2;
+  if (i + 1 < n) {
+    const float2 e = exp2_poly2(make_float2(x[i], x[i + 1]));
+    y[i] = e.x;
+    y[i + 1] = e.y;
+  } else if (i < n) {
+    y[i] = exp2_poly2(make_float2(x[i], 0.f)).x;
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_exp2_selftest(const float* x, float* y, int n, cudaStream_t stream) {
+  exp2_selftest_kernel<<<(n + 511) / 512, 256, 0, stream>>>(x, y, n);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_combine(const Problem& p, cudaStream_t stream) {
   dim3 grid(p.C, (p.R + kRowsPerBlock - 1) / kRowsPerBlock);

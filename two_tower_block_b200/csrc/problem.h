@@ -45,11 +45,13 @@ struct Problem {
   SplitRecord* records; // [C]
   unsigned* err_word;
   unsigned long long wait_limit_ns;
+  int variant;          // tcgen05 kernel: 0 = S/P aliasing in TMEM (default), 2 = transposed PV (head_dim 128)
 };
 
 // Host launchers (each returns the cudaError_t of its launch).
 cudaError_t launch_attn_mma_sync(const Problem& p, cudaStream_t stream);
 cudaError_t launch_combine(const Problem& p, cudaStream_t stream);
+cudaError_t launch_exp2_selftest(const float* x, float* y, int n, cudaStream_t stream);
 cudaError_t launch_wait_selftest(unsigned* err_word, unsigned long long limit_ns, cudaStream_t stream);
 
 struct TmaMaps {
@@ -57,6 +59,8 @@ struct TmaMaps {
 };
 cudaError_t launch_attn_tcgen05(const Problem& p, const TmaMaps& maps, cudaStream_t stream);
 bool tcgen05_key_tile_supported(int key_tile);
+cudaError_t launch_attn_pt(const Problem& p, const TmaMaps& maps, cudaStream_t stream);
+size_t attn_pt_smem_bytes();
 size_t attn_tcgen05_smem_bytes(int D);
 size_t attn_mma_sync_smem_bytes(int D);
 

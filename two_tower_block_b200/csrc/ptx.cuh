@@ -71,6 +71,30 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+// 2^x for a pair of arguments on the FMA and integer pipes (no MUFU), for x in
+// [-125, 127]; arguments below -125 are clamped there (2^-125 ~ 2.4e-38).
+// Range reduction x = j + f with j = round(x) taken by the 1.5 * 2^23 shifter and
+// |f| <= 1/2; 2^f by a degree-3 polynomial whose coefficients were fitted for
+// this library by iteratively reweighted least squares on the relative error
+// over [-1/2, 1/2] (max relative error 7.5e-5, float32 Horner evaluation); 2^j is
+// added to the exponent field.  The method is the classic table-free reduction
+// (J.-M. Muller, "Elementary Functions: Algorithms and Implementation", ch. 11).
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  x.x = fmaxf(x.x, -125.f);
+  x.y = fmaxf(x.y, -125.f);
+  const float kShift = 12582912.f;  // 1.5 * 2^23: adding it rounds to an integer in the low bits
+  const float2 t = __fadd2_rn(x, make_float2(kShift, kShift));
+  const float2 j = __fadd2_rn(t, make_float2(-kShift, -kShift));
+  const float2 f = __ffma2_rn(j, make_float2(-1.f, -1.f), x);
+  float2 q = __ffma2_rn(make_float2(0.05517115443944931f, 0.05517115443944931f), f,
+                        make_float2(0.2426101416349411f, 0.2426101416349411f));
+  q = __ffma2_rn(q, f, make_float2(0.6932609677314758f, 0.6932609677314758f));
+  q = __ffma2_rn(q, f, make_float2(0.9999281167984009f, 0.9999281167984009f));
+  // t's low bits hold j (two's complement); shifted by 23 they are j << 23
+  return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
+}
+
 // ---------------------------------------------------------------- mbarrier --
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
@@ -142,6 +166,12 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* m, 
       "%4, %5}], [%2];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(m)), "r"(bar), "r"(x), "r"(y), "r"(z)
       : "memory");
+}
+// Bring a tile into L2 only (no shared-memory destination, no completion signal).
+__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap* m, int x, int y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global [%0, {%1, %2}];" ::"l"(reinterpret_cast<uint64_t>(m)),
+               "r"(x), "r"(y)
+               : "memory");
 }
 // Make generic-proxy shared-memory writes visible to the async proxy (tensor core).
 __device__ __forceinline__ void fence_proxy_async_smem() {

@@ -31,7 +31,7 @@ EXPORTED_SYMBOLS = [
     "tt_block_attn_plan", "tt_block_attn_plan_destroy", "tt_block_attn_plan_get_info", "tt_block_attn",
     "tt_block_attn_block_causal", "tt_block_attn_host", "tt_block_attn_check", "tt_block_attn_profile",
     "tt_block_attn_profile_read", "tt_selftest_wait_timeout", "tt_debug_work_split", "tt_status_string",
-    "tt_last_error_detail", "tt_block_attn_noalloc",
+    "tt_last_error_detail", "tt_block_attn_noalloc", "tt_selftest_exp2",
 ]
 
 
@@ -73,6 +73,7 @@ def lib() -> ctypes.CDLL:
     L.tt_selftest_wait_timeout.argtypes = [i, i, vp]
     L.tt_debug_work_split.argtypes = [i, ip, i, ctypes.POINTER(ctypes.c_longlong), ip, ip]
     L.tt_block_attn_noalloc.argtypes = [ctypes.POINTER(Desc)] + [vp] * 10
+    L.tt_selftest_exp2.argtypes = [i, vp, vp, i]
     L.tt_status_string.argtypes = [i]
     L.tt_status_string.restype = ctypes.c_char_p
     L.tt_last_error_detail.argtypes = []
@@ -244,6 +245,15 @@ def block_attn_block_causal(q, k_ctx, v_ctx, k_blk, v_blk, block_size, scale=0.0
 
 def selftest_wait_timeout(device=0, timeout_us=20000, stream=None) -> int:
     return lib().tt_selftest_wait_timeout(int(device), int(timeout_us), _stream(stream))
+
+
+def selftest_exp2(x, device=0):
+    """The softmax's FMA-pipe exp2 evaluated on the device for float32 values x."""
+    import numpy as np
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    y = np.empty_like(x)
+    _check(lib().tt_selftest_exp2(int(device), x.ctypes.data, y.ctypes.data, x.size), "tt_selftest_exp2")
+    return y
 
 
 def work_split(tiles_per_unit, num_ctas):
