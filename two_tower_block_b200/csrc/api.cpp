@@ -159,7 +159,9 @@ tt::Problem base_problem(tt_plan_t plan) {
 tt_status_t launch_all(tt_plan_t plan, const tt::Problem& p, cudaStream_t s) {
   cudaError_t e;
   prof_mark(plan, 0, s, true);
-  if (plan->kernel == TT_KERNEL_TCGEN05) {
+  if (plan->kernel == TT_KERNEL_TCGEN05 && p.variant == 3) {
+    e = tt::launch_attn_2sm(p, s);
+  } else if (plan->kernel == TT_KERNEL_TCGEN05) {
     tt::TmaMaps maps;
     memset(&maps, 0, sizeof(maps));
     const uint64_t D = p.D;
@@ -266,13 +268,24 @@ tt_status_t tt_block_attn_plan(const tt_block_attn_desc* desc, int device, tt_pl
   if (P->kernel == TT_KERNEL_TCGEN05) {
     P->key_tile = tt::kTcgen05KeyTile;
     // tuning knobs: TT_TCGEN05_KEY_TILE=64 selects the two-buffer 64-key pipeline;
-    // TT_TCGEN05_VARIANT=2 selects the transposed-PV kernel for head_dim 128
+    // TT_TCGEN05_VARIANT=2 selects the transposed-PV kernel for head_dim 128,
+    // TT_TCGEN05_VARIANT=3 the 2-SM kernel (head_dim 128, 128 % g == 0)
     if (const char* kt = std::getenv("TT_TCGEN05_KEY_TILE")) {
       const int v = std::atoi(kt);
       if (tt::tcgen05_key_tile_supported(v)) P->key_tile = v;
     }
-    if (const char* kv = std::getenv("TT_TCGEN05_VARIANT")) P->variant = std::atoi(kv) == 2 ? 2 : 0;
+    if (const char* kv = std::getenv("TT_TCGEN05_VARIANT")) {
+      const int v = std::atoi(kv);
+      P->variant = (v == 2 || v == 3) ? v : 0;
+    }
+    if (P->variant == 3 && (!tt::attn_2sm_supported(d.head_dim, g) || P->key_tile != 128)) P->variant = 0;
     P->C = d.num_ctas > 0 ? d.num_ctas : P->sm_count;
+    if (P->variant == 3) {
+      // one range per cluster of two CTAs; by default as many as can be resident at once
+      const int clusters = tt::attn_2sm_max_clusters();
+      if (clusters <= 0) P->variant = 0;
+      else if (d.num_ctas <= 0) P->C = clusters;
+    }
   } else {
     P->key_tile = tt::kMmaSyncKeyTile;
     const int rb = (P->R + 63) / 64;

@@ -45,7 +45,8 @@ struct Problem {
   SplitRecord* records; // [C]
   unsigned* err_word;
   unsigned long long wait_limit_ns;
-  int variant;          // tcgen05 kernel: 0 = S/P aliasing in TMEM (default), 2 = transposed PV (head_dim 128)
+  int variant;          // tcgen05 kernel: 0 = S/P aliasing in TMEM (default), 2 = transposed PV,
+                        // 3 = 2-SM pairs (head_dim 128)
 };
 
 // Host launchers (each returns the cudaError_t of its launch).
@@ -60,6 +61,10 @@ struct TmaMaps {
 cudaError_t launch_attn_tcgen05(const Problem& p, const TmaMaps& maps, cudaStream_t stream);
 bool tcgen05_key_tile_supported(int key_tile);
 cudaError_t launch_attn_pt(const Problem& p, const TmaMaps& maps, cudaStream_t stream);
+// 2-SM kernel (cluster of two CTAs, one range per cluster): head_dim 128, 128 % g == 0
+bool attn_2sm_supported(int D, int g);
+int attn_2sm_max_clusters();
+cudaError_t launch_attn_2sm(const Problem& p, cudaStream_t stream);
 size_t attn_pt_smem_bytes();
 size_t attn_tcgen05_smem_bytes(int D);
 size_t attn_mma_sync_smem_bytes(int D);

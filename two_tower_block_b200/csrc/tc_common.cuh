@@ -49,15 +49,7 @@ __device__ __forceinline__ float tile_exp_store(const uint32_t* v, int count, fl
     for (int k = 0; k < 16; ++k) {
       const int c0 = 32 * ch + 2 * k;
       const float2 x = __ffma2_rn(make_float2(__uint_as_float(v[c0]), __uint_as_float(v[c0 + 1])), c2, nm2);
-      float a, b;
-      if ((k & 3) == 3) {  // one pair in four on the FMA pipe, the rest on MUFU
-        const float2 e = exp2_poly2(x);
-        a = e.x;
-        b = e.y;
-      } else {
-        a = fast_exp2(x.x);
-        b = fast_exp2(x.y);
-      }
+      float a = fast_exp2(x.x), b = fast_exp2(x.y);
       if (!kFull) {
         a = c0 < count ? a : 0.f;
         b = c0 + 1 < count ? b : 0.f;
@@ -83,15 +75,7 @@ __device__ __forceinline__ float tile_exp_pack(const uint32_t* v, int count, flo
   for (int k = 0; k < NK / 2; ++k) {
     const int c0 = 2 * k;
     const float2 x = __ffma2_rn(make_float2(__uint_as_float(v[c0]), __uint_as_float(v[c0 + 1])), c2, nm2);
-    float a, b;
-    if ((k & 3) == 3) {  // one pair in four on the FMA pipe, the rest on MUFU
-      const float2 e = exp2_poly2(x);
-      a = e.x;
-      b = e.y;
-    } else {
-      a = fast_exp2(x.x);
-      b = fast_exp2(x.y);
-    }
+    float a = fast_exp2(x.x), b = fast_exp2(x.y);
     if (!kFull) {
       a = c0 < count ? a : 0.f;
       b = c0 + 1 < count ? b : 0.f;
