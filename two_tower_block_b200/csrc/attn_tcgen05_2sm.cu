@@ -18,9 +18,12 @@
 //
 // Each CTA runs two softmax warpgroups that take alternate key tiles; each
 // has its own S buffer and O accumulator in TMEM (S_0 | S_1 | O_0 | O_1, 4 x 128
-// columns), its own running maximum and sum.  While one warpgroup works on
-// tile j the tensor cores compute S(j+1) for the other and P(j-1) V.  The two
-// partial softmax states of a row are merged exactly in the epilogue.
+// columns), two P buffers in shared memory, its own running maximum and sum.
+// The scores of tile j + 2 are computed as soon as tile j's scores have been
+// read into registers, so a warpgroup finds its next S ready when it finishes
+// a tile; with two P buffers it writes P(j) while P(j - 2) V may still run, and
+// waits for that product only when O must be rescaled.  The two partial
+// softmax states of a row are merged exactly in the epilogue.
 //
 // Synchronisation across the pair: the even CTA's MMA thread commits with
 // multicast to barriers in both CTAs; the odd CTA forwards its TMA completions
@@ -46,20 +49,20 @@ constexpr int kNK = 128;                       // keys per tile
 constexpr int kRowBytes = 128;                 // one 64-element bf16 half-row (swizzle atom width)
 constexpr int kHalf = 128 * kRowBytes;         // 16 KB: 128 rows x 64 elements
 constexpr int kQOff = 0;                       // Q: [2 d-halves][128 rows][128 B]      32 KB
-constexpr int kPOff = 2 * kHalf;               // P_w: [2 key-halves][128 rows][128 B]  2 x 32 KB
+constexpr int kPOff = 2 * kHalf;               // P[w][b]: [2 key-halves][128 rows][128 B]  4 x 32 KB
 constexpr int kPBytes = 2 * kHalf;
-constexpr int kRingOff = kPOff + 2 * kPBytes;  // K/V ring
+constexpr int kRingOff = kPOff + 4 * kPBytes;  // K/V ring
 constexpr int kEntryBytes = 16384;             // K: [2 d-halves][64 keys][128 B]; V: [128 keys][128 B]
-constexpr int kStages = 7;
+constexpr int kStages = 4;
 constexpr int kMiscOff = kRingOff + kStages * kEntryBytes;
 constexpr float kRescaleThreshold = 8.0f;
 constexpr int kCtrlRegs = 80, kSoftmaxRegs = 200;
 static_assert(4 * 32 * kCtrlRegs + 8 * 32 * kSoftmaxRegs <= kThreads * 168, "register split");
 
 struct Bars {
-  uint64_t q_full, q_ready, q_empty, tail, drain, epi;
+  uint64_t q_full, q_ready, q_empty, tail, drain, epi, epi_done;
   uint64_t kv_full[kStages], kv_ready[kStages], kv_empty[kStages];
-  uint64_t s_full[2], s_free[2], p_full[2], pv_done[2];
+  uint64_t s_full[2], s_free[2], p_full[2], pv_done[2][2];   // pv_done[warpgroup][P buffer]
   uint64_t o_full, o_empty;
 };
 
@@ -69,7 +72,7 @@ struct Misc {
   int abort_flag;
   long long T, start, end;
   Unit first;
-  float ml[2][2][2][128];   // [segment parity][warpgroup][m or l][row]: epilogue exchange
+  float ml[2][2][128];      // [warpgroup][m or l][row]: epilogue exchange
 };
 
 constexpr int kSmemBytes = kMiscOff + (int)sizeof(Misc);
@@ -77,16 +80,21 @@ static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 __device__ __forceinline__ uint64_t add16(uint64_t desc, uint32_t byte_off) { return desc + (uint64_t)(byte_off >> 4); }
 
-// ring entries of a segment with n tiles, in the order the MMA consumes them:
-// K0, K1, V0, K2, V1, ..., K(n-1), V(n-2), V(n-1)
+// Ring entries of a segment with n tiles, in the order the MMA consumes them: the scores
+// of tile j + 2 are computed as soon as tile j's scores have been read, before P(j) V:
+// K0, K1, K2, V0, K3, V1, ..., K(n-1), V(n-3), V(n-2), V(n-1)
 __device__ __forceinline__ void entry_to_tile(int e, int n, int& j, int& kv) {
   if (e == 0) { j = 0; kv = 0; }
-  else if (e == 2 * n - 1) { j = n - 1; kv = 1; }
-  else if (e & 1) { j = (e + 1) >> 1; kv = 0; }
-  else { j = (e >> 1) - 1; kv = 1; }
+  else if (e == 1) { j = n == 1 ? 0 : 1; kv = n == 1 ? 1 : 0; }
+  else if (e <= 2 * n - 3) {
+    if (e & 1) { j = (e - 3) >> 1; kv = 1; }
+    else { j = (e >> 1) + 1; kv = 0; }
+  } else { j = e - n; kv = 1; }   // e = 2n-2 -> V(n-2), e = 2n-1 -> V(n-1)
 }
-__device__ __forceinline__ uint32_t entry_k(int j) { return j == 0 ? 0u : (uint32_t)(2 * j - 1); }
-__device__ __forceinline__ uint32_t entry_v(int j, int n) { return j == n - 1 ? (uint32_t)(2 * n - 1) : (uint32_t)(2 * j + 2); }
+__device__ __forceinline__ uint32_t entry_k(int t) { return t < 2 ? (uint32_t)t : (uint32_t)(2 * t - 2); }
+__device__ __forceinline__ uint32_t entry_v(int j, int n) {
+  return j + 2 < n ? (uint32_t)(2 * j + 3) : (uint32_t)(n + j);
+}
 
 // P row of one warp lane to shared memory: weights exp2(s * c - m_ref) of the 128 keys,
 // rounded to bf16, written as 16-byte chunks in the 128-byte swizzled K-major layout
@@ -145,6 +153,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     mbar_init(bar(bars->tail), 1);
     mbar_init(bar(bars->drain), 1);
     mbar_init(bar(bars->epi), 256);
+    mbar_init(bar(bars->epi_done), 256);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(bar(bars->kv_full[s]), 1);
       mbar_init(bar(bars->kv_ready[s]), 2);
@@ -154,7 +163,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       mbar_init(bar(bars->s_full[w]), 1);
       mbar_init(bar(bars->s_free[w]), 8);   // 4 warps in each CTA
       mbar_init(bar(bars->p_full[w]), 8);
-      mbar_init(bar(bars->pv_done[w]), 1);
+      mbar_init(bar(bars->pv_done[w][0]), 1);
+      mbar_init(bar(bars->pv_done[w][1]), 1);
     }
     mbar_init(bar(bars->o_full), 1);
     mbar_init(bar(bars->o_empty), 16);      // 8 softmax warps in each CTA
@@ -319,7 +329,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         tc_commit2_both(bar(bars->s_full[g & 1]));
         tc_commit2_both(bar(bars->kv_empty[e % kStages]));
       };
-      // the S buffer of tile g was last used by tile g - 2: its softmax must have loaded it
+      // the S buffer of tile g was last used by tile g - 2: its softmax must have read it
       auto s_buffer_free = [&](uint32_t g) {
         if (g < 2) return true;
         return mbar_wait_cluster(bar(bars->s_free[g & 1]), ((g >> 1) & 1) ^ 1, wc);
@@ -329,19 +339,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int n = sg.hi - sg.lo;
         ok = mbar_wait_cluster(bar(bars->q_ready), q_it & 1, wc);
         ++q_it;
-        if (ok) ok = s_buffer_free(G);
-        if (ok) ok = ring_wait(it + entry_k(0));
-        if (!ok) break;
-        tc_fence_after();
-        issue_s(G, it + entry_k(0), round16(tile_keys(p, x, sg.lo).count));
+        // S of tile t of the segment; Q is released after the segment's last S
+        auto s_tile = [&](int t) {
+          const uint32_t g = G + t;
+          if (!s_buffer_free(g)) return false;
+          if (!ring_wait(it + entry_k(t))) return false;
+          tc_fence_after();
+          issue_s(g, it + entry_k(t), round16(tile_keys(p, x, sg.lo + t).count));
+          if (t == n - 1) tc_commit2_both(bar(bars->q_empty));
+          return true;
+        };
+        for (int t = 0; t < 2 && t < n && ok; ++t) ok = s_tile(t);
         for (int j = 0; j < n && ok; ++j) {
           const uint32_t g = G + j;
-          if (j + 1 < n) {
-            ok = s_buffer_free(g + 1);
-            if (ok) ok = ring_wait(it + entry_k(j + 1));
+          if (j + 2 < n) {
+            ok = s_tile(j + 2);   // waits until tile j's scores have been read
             if (!ok) break;
-            tc_fence_after();
-            issue_s(g + 1, it + entry_k(j + 1), round16(tile_keys(p, x, sg.lo + j + 1).count));
           }
           const uint32_t ev = it + entry_v(j, n);
           ok = mbar_wait_cluster(bar(bars->p_full[g & 1]), (g >> 1) & 1, wc);
@@ -350,17 +363,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           if (!ok) break;
           tc_fence_after();
           const int nv = round16(tile_keys(p, x, sg.lo + j).count);
-          const uint64_t pd = add16(pdesc, (g & 1) * kPBytes);
+          const uint32_t pb = (g & 1) * 2 + ((g >> 1) & 1);   // P[warpgroup][buffer]
+          const uint64_t pd = add16(pdesc, pb * kPBytes);
           const uint64_t vd = add16(vdesc, (ev % kStages) * kEntryBytes);
           for (int kk = 0; kk < nv / 16; ++kk)
             tc_mma2_ss(tmem + 256 + 128 * (g & 1), add16(pd, (kk >> 2) * kHalf + (kk & 3) * 32),
                        add16(vd, kk * 16 * kRowBytes), idesc_pv, (j >= 2 || kk > 0) ? 1u : 0u);
-          tc_commit2_both(bar(bars->pv_done[g & 1]));
+          tc_commit2_both(bar(bars->pv_done[g & 1][(g >> 1) & 1]));
           tc_commit2_both(bar(bars->kv_empty[ev % kStages]));
         }
         if (!ok) break;
         tc_commit2_both(bar(bars->o_full));
-        tc_commit2_both(bar(bars->q_empty));
         it += 2 * n;
         G += n;
         ++seg_cnt;
@@ -379,7 +392,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
     const uint32_t s_addr = tmem + lane_off + 128 * w;
     const uint32_t o_base = tmem + lane_off + 256;   // O_0 at +0, O_1 at +128
-    uint8_t* prow = smem + kPOff + w * kPBytes + lr * kRowBytes;
+    uint8_t* prow0 = smem + kPOff + 2 * w * kPBytes + lr * kRowBytes;   // P[w][0]; P[w][1] follows
     uint32_t G = 0, seg_cnt = 0;
     bool ok = true;
     Unit x = ms->first;
@@ -405,18 +418,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (lane == 0) arrive_even(bars->s_free[w]);   // S may be overwritten by tile g + 2
         const float mx = (full ? tile_row_max<kNK, true>(v, count) : tile_row_max<kNK, false>(v, count)) * p.scale_log2;
-        // The PV of this warpgroup's previous tile (g - 2) was issued before S(g), so it has
-        // completed by now (the tensor pipe runs in order): O_w and P_w are free.
-        if (g >= 2) {
-          ok = mbar_wait(bar(bars->pv_done[w]), ((g >> 1) & 1) ^ 1, wc);
-          if (!ok) break;
-          tc_fence_after();
-        }
+        const uint32_t b = (g >> 1) & 1;   // P buffer of this tile; tile g - 2 used the other one
         if (first) {
           m_w = mx;  // O_w is overwritten by this warpgroup's first PV of the segment
         } else {
           const bool need = mx > m_w + kRescaleThreshold;
           if (__any_sync(0xffffffffu, need)) {
+            // O_w must hold P(g-2) V before it is rescaled
+            ok = mbar_wait(bar(bars->pv_done[w][b ^ 1]), ((g - 2) >> 2) & 1, wc);
+            if (!ok) break;
+            tc_fence_after();
             const float alpha = need ? fast_exp2(m_w - mx) : 1.f;
             if (need) {
               m_w = mx;
@@ -434,6 +445,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             tc_wait_st();
           }
         }
+        // P buffer b was last read by the PV of tile g - 4
+        if (g >= 4) {
+          ok = mbar_wait(bar(bars->pv_done[w][b]), ((g >> 2) & 1) ^ 1, wc);
+          if (!ok) break;
+          tc_fence_after();
+        }
+        uint8_t* prow = prow0 + b * kPBytes;
         l_w += full ? exp_to_smem<true>(v, count, p.scale_log2, m_w, prow, lr)
                     : exp_to_smem<false>(v, count, p.scale_log2, m_w, prow, lr);
         fence_proxy_async_smem();
@@ -448,13 +466,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (!ok) break;
       tc_fence_after();
       const int par = seg_cnt & 1;
-      ms->ml[par][w][0][lr] = first ? -INFINITY : m_w;
-      ms->ml[par][w][1][lr] = first ? 0.f : l_w;
+      // the previous segment's exchange must have been read by every thread of the CTA
+      if (seg_cnt > 0) {
+        ok = mbar_wait(bar(bars->epi_done), par ^ 1, wc);
+        if (!ok) break;
+      }
+      ms->ml[w][0][lr] = first ? -INFINITY : m_w;
+      ms->ml[w][1][lr] = first ? 0.f : l_w;
       mbar_arrive(bar(bars->epi));
       ok = mbar_wait(bar(bars->epi), par, wc);
       if (!ok) break;
-      const float mA = ms->ml[par][0][0][lr], lA = ms->ml[par][0][1][lr];
-      const float mB = ms->ml[par][1][0][lr], lB = ms->ml[par][1][1][lr];
+      const float mA = ms->ml[0][0][lr], lA = ms->ml[0][1][lr];
+      const float mB = ms->ml[1][0][lr], lB = ms->ml[1][1][lr];
+      mbar_arrive(bar(bars->epi_done));
       const bool hasA = n >= 1 && ((G & 1) == 0 || n >= 2);   // warpgroup 0 had a tile
       const bool hasB = n >= 1 && ((G & 1) == 1 || n >= 2);   // warpgroup 1 had a tile
       const float m = fmaxf(hasA ? mA : -INFINITY, hasB ? mB : -INFINITY);
