@@ -49,6 +49,7 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--num-ctas", type=int, default=0, help="work ranges (0: the plan's choice)")
     return ap.parse_args()
 
 
@@ -261,7 +262,7 @@ def run_native(args):
     if w.kind == "decode":
         lens = torch.from_numpy(inp.ctx_lens).to(dev)
         plan = ops.Plan(w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_size, ctx_capacity=w.ctx,
-                        kernel=kernel, device=local)
+                        kernel=kernel, num_ctas=args.num_ctas, device=local)
         out = torch.empty((w.batch, w.block_size, w.num_q_heads, w.head_dim), dtype=torch.float32, device=dev)
         lse = torch.empty((w.batch, w.num_q_heads, w.block_size), dtype=torch.float32, device=dev)
 
@@ -270,7 +271,7 @@ def run_native(args):
             plan.block_attn(c[0], c[1], c[2], c[3], c[4], lens, out=out, lse=lse)
     else:
         plan = ops.Plan(w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_size, seq_len=w.seq_len,
-                        kernel=kernel, device=local)
+                        kernel=kernel, num_ctas=args.num_ctas, device=local)
         out = torch.empty((w.batch, w.seq_len, w.num_q_heads, w.head_dim), dtype=torch.float32, device=dev)
         lse = torch.empty((w.batch, w.num_q_heads, w.seq_len), dtype=torch.float32, device=dev)
 
@@ -333,7 +334,7 @@ def run_native(args):
     e2e = None
     if w.kind == "decode" and not args.no_e2e:
         hplan = ops.Plan(w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_size, ctx_capacity=w.ctx,
-                         kernel=kernel, host_io=True, device=local)
+                         kernel=kernel, num_ctas=args.num_ctas, host_io=True, device=local)
 
         def pinned(bits):
             return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).pin_memory()
