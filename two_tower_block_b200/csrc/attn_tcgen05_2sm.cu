@@ -25,10 +25,15 @@
 // waits for that product only when O must be rescaled.  The two partial
 // softmax states of a row are merged exactly in the epilogue.
 //
+// The MMA thread issues S(j+2) interleaved, instruction by instruction, with P(j-1) V
+// (the other warpgroup's product), so that two independent accumulator chains are in
+// flight (the ring order below follows).
+//
 // Synchronisation across the pair: the even CTA's MMA thread commits with
-// multicast to barriers in both CTAs; the odd CTA forwards its TMA completions
-// and the arrivals of its softmax warps to the even CTA's barriers (remote
-// mbarrier arrive).  No TMA multicast is used.  Every wait is bounded
+// multicast to barriers in both CTAs.  The odd CTA's TMA completions and softmax
+// arrivals land on its own barriers and are forwarded to the even CTA's by
+// otherwise idle warps (remote mbarrier arrive), so no softmax warp pays for a
+// cluster-scope release.  No TMA multicast is used.  Every wait is bounded
 // (ptx.cuh); on a timeout the CTA raises the error word and both CTAs still
 // meet at the final cluster barrier before TMEM is released.
 #include <algorithm>
@@ -64,6 +69,7 @@ struct Bars {
   uint64_t kv_full[kStages], kv_ready[kStages], kv_empty[kStages];
   uint64_t s_full[2], s_free[2], p_full[2], pv_done[2][2];   // pv_done[warpgroup][P buffer]
   uint64_t o_full, o_empty;
+  uint64_t o_done[2];   // odd CTA: its warpgroup w has read O (forwarded to the even CTA's o_empty)
 };
 
 struct Misc {
@@ -80,20 +86,20 @@ static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 __device__ __forceinline__ uint64_t add16(uint64_t desc, uint32_t byte_off) { return desc + (uint64_t)(byte_off >> 4); }
 
-// Ring entries of a segment with n tiles, in the order the MMA consumes them: the scores
-// of tile j + 2 are computed as soon as tile j's scores have been read, before P(j) V:
-// K0, K1, K2, V0, K3, V1, ..., K(n-1), V(n-3), V(n-2), V(n-1)
+// Ring entries of a segment with n tiles, in the order the MMA consumes them.  The MMA
+// thread issues S(j+2) interleaved, instruction by instruction, with P(j-1) V (the other
+// warpgroup's product), so that two independent accumulator chains are always in flight:
+// K0, K1, K2, (K3 V0), (K4 V1), ..., (K(n-1) V(n-4)), V(n-3), V(n-2), V(n-1)
 __device__ __forceinline__ void entry_to_tile(int e, int n, int& j, int& kv) {
-  if (e == 0) { j = 0; kv = 0; }
-  else if (e == 1) { j = n == 1 ? 0 : 1; kv = n == 1 ? 1 : 0; }
-  else if (e <= 2 * n - 3) {
-    if (e & 1) { j = (e - 3) >> 1; kv = 1; }
-    else { j = (e >> 1) + 1; kv = 0; }
-  } else { j = e - n; kv = 1; }   // e = 2n-2 -> V(n-2), e = 2n-1 -> V(n-1)
+  if (e < min(n, 3)) { j = e; kv = 0; }
+  else if (n >= 3 && e <= 2 * n - 4) {
+    if (e & 1) { j = (e + 3) >> 1; kv = 0; }
+    else { j = (e - 4) >> 1; kv = 1; }
+  } else { j = e - n; kv = 1; }
 }
-__device__ __forceinline__ uint32_t entry_k(int t) { return t < 2 ? (uint32_t)t : (uint32_t)(2 * t - 2); }
-__device__ __forceinline__ uint32_t entry_v(int j, int n) {
-  return j + 2 < n ? (uint32_t)(2 * j + 3) : (uint32_t)(n + j);
+__device__ __forceinline__ uint32_t entry_k(int t) { return t <= 2 ? (uint32_t)t : (uint32_t)(2 * t - 3); }
+__device__ __forceinline__ uint32_t entry_v(int i, int n) {
+  return i <= n - 4 ? (uint32_t)(2 * i + 4) : (uint32_t)(n + i);
 }
 
 // P row of one warp lane to shared memory: weights exp2(s * c - m_ref) of the 128 keys,
@@ -139,11 +145,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const bool aligned = (sbase & 1023u) == 0;   // the swizzled layouts need a 1024-byte aligned base
   const uint32_t q_s = sbase + kQOff, p_s = sbase + kPOff, ring_s = sbase + kRingOff;
   auto bar = [&](const uint64_t& b) { return smem_u32(&b); };
-  // arrive on a barrier of the even CTA (locally there, remotely from the odd CTA)
-  auto arrive_even = [&](const uint64_t& b) {
-    if (rank == 0) mbar_arrive(bar(b));
-    else mbar_arrive_remote(mapa_shared(bar(b), 0));
-  };
+  // Softmax warps arrive on barriers of their own CTA only: a cluster-scope release
+  // costs a softmax warp a thousand cycles or more, so the odd CTA's arrivals are
+  // forwarded to the even CTA by otherwise idle warps (see the forwarders below).
 
   // ---------------------------------------------------------------- setup --
   if (tid == 0) {
@@ -161,13 +165,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     for (int w = 0; w < 2; ++w) {
       mbar_init(bar(bars->s_full[w]), 1);
-      mbar_init(bar(bars->s_free[w]), 8);   // 4 warps in each CTA
-      mbar_init(bar(bars->p_full[w]), 8);
+      // even CTA: its 4 warps + one forwarded arrival for the odd CTA's 4; odd CTA: its 4 warps
+      mbar_init(bar(bars->s_free[w]), rank == 0 ? 5 : 4);
+      mbar_init(bar(bars->p_full[w]), rank == 0 ? 5 : 4);
+      mbar_init(bar(bars->o_done[w]), 4);
       mbar_init(bar(bars->pv_done[w][0]), 1);
       mbar_init(bar(bars->pv_done[w][1]), 1);
     }
     mbar_init(bar(bars->o_full), 1);
-    mbar_init(bar(bars->o_empty), 16);      // 8 softmax warps in each CTA
+    mbar_init(bar(bars->o_empty), 10);      // even CTA: 8 softmax warps + 2 forwarded (odd warpgroups)
     ms->abort_flag = aligned ? 0 : 1;
     if (!aligned) raise_error(p.err_word, kErrInternal);
     fence_barrier_init();
@@ -277,24 +283,40 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         mbar_wait(rank == 0 ? bar(bars->kv_ready[j % kStages]) : bar(bars->kv_full[j % kStages]),
                   (j / kStages) & 1, dw);
     }
-  } else if ((warp == 2 || warp == 3) && rank == 1 && have_work) {
-    // ======================================= odd CTA: forward TMA completions ==
+  } else if (warp >= 1 && warp <= 3 && rank == 1 && have_work) {
+    // ===================================== odd CTA: forward completions to the even CTA ==
+    // warp 2: the TMA completions of Q and of every K/V ring entry, in the order the
+    // producer issued them; warp 1 (warp 3): the arrivals of softmax warpgroup 0 (1),
+    // tile by tile (S read, P written) and O read at the end of each segment.
     if (lane == 0) {
-      uint32_t it = 0, q_it = 0;
+      uint32_t it = 0, q_it = 0, G = 0, seg_cnt = 0;
+      const int w = warp == 1 ? 0 : 1;
       bool ok = true;
       Unit x = ms->first;
       for (; ok;) {
         const Segment sg = segment_of(x, start, end, c);
         const int n = sg.hi - sg.lo;
-        if (warp == 3) {
+        if (warp == 2) {
           ok = mbar_wait(bar(bars->q_full), q_it & 1, wc);
           if (ok) mbar_arrive_remote(mapa_shared(bar(bars->q_ready), 0));
           ++q_it;
-        } else {
           for (int e = 0; e < 2 * n && ok; ++e, ++it) {
             ok = mbar_wait(bar(bars->kv_full[it % kStages]), (it / kStages) & 1, wc);
             if (ok) mbar_arrive_remote(mapa_shared(bar(bars->kv_ready[it % kStages]), 0));
           }
+        } else {
+          for (int j = 0; j < n && ok; ++j) {
+            const uint32_t g = G + j;
+            if ((int)(g & 1) != w) continue;
+            ok = mbar_wait(bar(bars->s_free[w]), (g >> 1) & 1, wc);
+            if (ok) mbar_arrive_remote(mapa_shared(bar(bars->s_free[w]), 0));
+            if (ok) ok = mbar_wait(bar(bars->p_full[w]), (g >> 1) & 1, wc);
+            if (ok) mbar_arrive_remote(mapa_shared(bar(bars->p_full[w]), 0));
+          }
+          if (ok) ok = mbar_wait(bar(bars->o_done[w]), seg_cnt & 1, wc);
+          if (ok) mbar_arrive_remote(mapa_shared(bar(bars->o_empty), 0));
+          G += n;
+          ++seg_cnt;
         }
         if (!ok || sg.last) break;
         x = make_unit(p, x.u + 1, x.Tu + x.tiles);
@@ -316,19 +338,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       auto ring_wait = [&](uint32_t e) {
         return mbar_wait_cluster(bar(bars->kv_ready[e % kStages]), (e / kStages) & 1, wc);
       };
-      // S of tile g (buffer g & 1) from ring entry e
-      auto issue_s = [&](uint32_t g, uint32_t e, int nk) {
-        const uint32_t idesc = idesc_s0 | ((uint32_t)(nk >> 3) << 17);
-        const uint64_t kd = add16(kdesc, (e % kStages) * kEntryBytes);
-#pragma unroll
-        for (int kk = 0; kk < kD / 16; ++kk) {
-          const uint32_t qo = (kk >> 2) * kHalf + (kk & 3) * 32;
-          const uint32_t ko = (kk >> 2) * (64 * kRowBytes) + (kk & 3) * 32;
-          tc_mma2_ss(tmem + 128 * (g & 1), add16(qdesc, qo), add16(kd, ko), idesc, kk > 0);
-        }
-        tc_commit2_both(bar(bars->s_full[g & 1]));
-        tc_commit2_both(bar(bars->kv_empty[e % kStages]));
-      };
       // the S buffer of tile g was last used by tile g - 2: its softmax must have read it
       auto s_buffer_free = [&](uint32_t g) {
         if (g < 2) return true;
@@ -339,39 +348,57 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int n = sg.hi - sg.lo;
         ok = mbar_wait_cluster(bar(bars->q_ready), q_it & 1, wc);
         ++q_it;
-        // S of tile t of the segment; Q is released after the segment's last S
-        auto s_tile = [&](int t) {
-          const uint32_t g = G + t;
-          if (!s_buffer_free(g)) return false;
-          if (!ring_wait(it + entry_k(t))) return false;
+        // One step: S of tile t (when t < n) and P V of tile i (when 0 <= i), issued
+        // interleaved.  Q is released after the segment's last S.
+        auto step = [&](int t, int i) -> bool {
+          const bool has_s = t < n, has_pv = i >= 0;
+          if (!has_s && !has_pv) return true;
+          const uint32_t gs = G + t, gp = G + i;
+          uint32_t ek = 0, ev = 0;
+          if (has_s) {
+            if (!s_buffer_free(gs)) return false;
+            ek = it + entry_k(t);
+            if (!ring_wait(ek)) return false;
+          }
+          if (has_pv) {
+            if (!mbar_wait_cluster(bar(bars->p_full[gp & 1]), (gp >> 1) & 1, wc)) return false;
+            ev = it + entry_v(i, n);
+            if (!ring_wait(ev)) return false;
+            if (i == 0 && !mbar_wait_cluster(bar(bars->o_empty), (seg_cnt & 1) ^ 1, wc)) return false;
+          }
           tc_fence_after();
-          issue_s(g, it + entry_k(t), round16(tile_keys(p, x, sg.lo + t).count));
-          if (t == n - 1) tc_commit2_both(bar(bars->q_empty));
+          const int nk = has_s ? round16(tile_keys(p, x, sg.lo + t).count) : 0;
+          const int npv = has_pv ? round16(tile_keys(p, x, sg.lo + i).count) / 16 : 0;
+          const uint32_t idesc_s = idesc_s0 | ((uint32_t)(nk >> 3) << 17);
+          const uint64_t kd = add16(kdesc, (ek % kStages) * kEntryBytes);
+          const uint64_t pd = add16(pdesc, ((gp & 1) * 2 + ((gp >> 1) & 1)) * kPBytes);   // P[warpgroup][buffer]
+          const uint64_t vd = add16(vdesc, (ev % kStages) * kEntryBytes);
+          const uint32_t s_acc = tmem + 128 * (gs & 1), o_acc = tmem + 256 + 128 * (gp & 1);
+          const uint32_t pv_acc0 = i >= 2 ? 1u : 0u;   // O_w starts at this warpgroup's first tile
+#pragma unroll
+          for (int kk = 0; kk < kD / 16; ++kk) {
+            if (has_s)
+              tc_mma2_ss(s_acc, add16(qdesc, (kk >> 2) * kHalf + (kk & 3) * 32),
+                         add16(kd, (kk >> 2) * (64 * kRowBytes) + (kk & 3) * 32), idesc_s, kk > 0);
+            if (kk < npv)
+              tc_mma2_ss(o_acc, add16(pd, (kk >> 2) * kHalf + (kk & 3) * 32), add16(vd, kk * 16 * kRowBytes),
+                         idesc_pv, kk > 0 ? 1u : pv_acc0);
+          }
+          if (has_s) {
+            tc_commit2_both(bar(bars->s_full[gs & 1]));
+            tc_commit2_both(bar(bars->kv_empty[ek % kStages]));
+            if (t == n - 1) tc_commit2_both(bar(bars->q_empty));
+          }
+          if (has_pv) {
+            tc_commit2_both(bar(bars->pv_done[gp & 1][(gp >> 1) & 1]));
+            tc_commit2_both(bar(bars->kv_empty[ev % kStages]));
+          }
           return true;
         };
-        for (int t = 0; t < 2 && t < n && ok; ++t) ok = s_tile(t);
-        for (int j = 0; j < n && ok; ++j) {
-          const uint32_t g = G + j;
-          if (j + 2 < n) {
-            ok = s_tile(j + 2);   // waits until tile j's scores have been read
-            if (!ok) break;
-          }
-          const uint32_t ev = it + entry_v(j, n);
-          ok = mbar_wait_cluster(bar(bars->p_full[g & 1]), (g >> 1) & 1, wc);
-          if (ok) ok = ring_wait(ev);
-          if (ok && j == 0) ok = mbar_wait_cluster(bar(bars->o_empty), (seg_cnt & 1) ^ 1, wc);
-          if (!ok) break;
-          tc_fence_after();
-          const int nv = round16(tile_keys(p, x, sg.lo + j).count);
-          const uint32_t pb = (g & 1) * 2 + ((g >> 1) & 1);   // P[warpgroup][buffer]
-          const uint64_t pd = add16(pdesc, pb * kPBytes);
-          const uint64_t vd = add16(vdesc, (ev % kStages) * kEntryBytes);
-          for (int kk = 0; kk < nv / 16; ++kk)
-            tc_mma2_ss(tmem + 256 + 128 * (g & 1), add16(pd, (kk >> 2) * kHalf + (kk & 3) * 32),
-                       add16(vd, kk * 16 * kRowBytes), idesc_pv, (j >= 2 || kk > 0) ? 1u : 0u);
-          tc_commit2_both(bar(bars->pv_done[g & 1][(g >> 1) & 1]));
-          tc_commit2_both(bar(bars->kv_empty[ev % kStages]));
-        }
+        ok = step(0, -1);
+        if (ok && n > 1) ok = step(1, -1);
+        for (int j = 0; j < n && ok; ++j) ok = step(j + 2, j - 1);
+        if (ok) ok = step(n, n - 1);
         if (!ok) break;
         tc_commit2_both(bar(bars->o_full));
         it += 2 * n;
@@ -416,7 +443,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         tc_wait_ld();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) arrive_even(bars->s_free[w]);   // S may be overwritten by tile g + 2
+        if (lane == 0) mbar_arrive(bar(bars->s_free[w]));   // S may be overwritten by tile g + 2
         const float mx = (full ? tile_row_max<kNK, true>(v, count) : tile_row_max<kNK, false>(v, count)) * p.scale_log2;
         const uint32_t b = (g >> 1) & 1;   // P buffer of this tile; tile g - 2 used the other one
         if (first) {
@@ -457,7 +484,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) arrive_even(bars->p_full[w]);
+        if (lane == 0) mbar_arrive(bar(bars->p_full[w]));
         first = false;
       }
       if (!ok) break;
@@ -497,7 +524,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         if (cc == 3) {
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) arrive_even(bars->o_empty);  // O read: the next segment may overwrite it
+          if (lane == 0) mbar_arrive(rank == 0 ? bar(bars->o_empty) : bar(bars->o_done[w]));  // O read
         }
         if (r < p.R) {
           float* dst = out_row(p, x, sg, r, kD) + col;
