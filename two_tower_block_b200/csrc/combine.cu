@@ -14,7 +14,7 @@ namespace {
 
 constexpr int kRowsPerBlock = 8;   // one warp per row
 constexpr int kThreads = 256;
-constexpr int kMaxSegInRegs = 32;  // segments whose weight one lane keeps (lane s holds segment s)
+constexpr int kGroup = 8;          // segments whose rows a warp loads together
 
 template <int D>
 __global__ void __launch_bounds__(kThreads) combine_kernel(const Problem p) {
@@ -28,49 +28,58 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const Problem p) {
   const int nseg = rec.last_range - c + 1;
   constexpr int V = D / 32;  // columns per lane
   auto slot_of = [&](int s) { return s == 0 ? 2 * c + rec.first_which : 2 * (c + s); };
-  // weights: lane s holds segment s (segments beyond 32 are folded in a second sweep)
-  float M = -INFINITY;
-  for (int s = lane; s < nseg; s += 32) M = fmaxf(M, p.part_lse[(size_t)slot_of(s) * p.R + r]);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  auto load_row = [&](int s, float* a) {
+    const float* src = p.part_o + ((size_t)slot_of(s) * p.R + r) * D + lane * V;
+    if constexpr (V == 4) {
+      const float4 t = __ldcg(reinterpret_cast<const float4*>(src));
+      a[0] = t.x; a[1] = t.y; a[2] = t.z; a[3] = t.w;
+    } else {
+      const float2 t = __ldcg(reinterpret_cast<const float2*>(src));
+      a[0] = t.x; a[1] = t.y;
+    }
+  };
   float acc[V];
 #pragma unroll
   for (int v = 0; v < V; ++v) acc[v] = 0.f;
-  float wsum = 0.f;
-  for (int s0 = 0; s0 < nseg; s0 += kMaxSegInRegs) {
-    const int s = s0 + lane;
-    const float w_lane = s < nseg ? expf(p.part_lse[(size_t)slot_of(s) * p.R + r] - M) : 0.f;
+  float M = -INFINITY, wsum = 0.f;
+  // segments in sweeps of 32 (lane s holds segment s0 + s): the lse values and the first
+  // kGroup rows are requested together, the rest kGroup at a time
+  for (int s0 = 0; s0 < nseg; s0 += 32) {
+    const int n = min(32, nseg - s0);
+    const float lse_lane = lane < n ? __ldcg(p.part_lse + (size_t)slot_of(s0 + lane) * p.R + r) : -INFINITY;
+    float a[kGroup][V];
+#pragma unroll
+    for (int u = 0; u < kGroup; ++u)
+      if (u < n) load_row(s0 + u, a[u]);
+    float Ms = lse_lane;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) Ms = fmaxf(Ms, __shfl_xor_sync(0xffffffffu, Ms, o));
+    // fold this sweep into the running (M, wsum, acc)
+    const float Mn = fmaxf(M, Ms);
+    const float scale_old = M == -INFINITY ? 0.f : expf(M - Mn);
+    wsum *= scale_old;
+#pragma unroll
+    for (int v = 0; v < V; ++v) acc[v] *= scale_old;
+    M = Mn;
+    const float w_lane = lane < n ? expf(lse_lane - M) : 0.f;
     float ws = w_lane;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) ws += __shfl_xor_sync(0xffffffffu, ws, o);
     wsum += ws;
-    const int n = min(kMaxSegInRegs, nseg - s0);
-    // four segments' rows in flight per step
-    for (int k = 0; k < n; k += 4) {
-      float a[4][V];
-      float w[4];
+    for (int k = 0; k < n; k += kGroup) {
+      if (k > 0) {
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        w[u] = __shfl_sync(0xffffffffu, w_lane, (k + u) & 31);
-        if (k + u < n) {
-          const float* src = p.part_o + ((size_t)slot_of(s0 + k + u) * p.R + r) * D + lane * V;
-          if constexpr (V == 4) {
-            const float4 t = __ldcg(reinterpret_cast<const float4*>(src));
-            a[u][0] = t.x; a[u][1] = t.y; a[u][2] = t.z; a[u][3] = t.w;
-          } else {
-            const float2 t = __ldcg(reinterpret_cast<const float2*>(src));
-            a[u][0] = t.x; a[u][1] = t.y;
-          }
-        } else {
-          w[u] = 0.f;
-#pragma unroll
-          for (int v = 0; v < V; ++v) a[u][v] = 0.f;
-        }
+        for (int u = 0; u < kGroup; ++u)
+          if (k + u < n) load_row(s0 + k + u, a[u]);
       }
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
+      for (int u = 0; u < kGroup; ++u) {
+        const float w = __shfl_sync(0xffffffffu, w_lane, (k + u) & 31);
+        if (k + u < n) {
 #pragma unroll
-        for (int v = 0; v < V; ++v) acc[v] = fmaf(w[u], a[u][v], acc[v]);
+          for (int v = 0; v < V; ++v) acc[v] = fmaf(w, a[u][v], acc[v]);
+        }
+      }
     }
   }
   const float inv = 1.f / wsum;
