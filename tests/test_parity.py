@@ -98,6 +98,18 @@ def test_split_count_invariance(kernel, num_ctas):
     assert_parity(lse, rl, f"C={num_ctas} lse")
 
 
+@pytest.mark.parametrize("kernel", KERNELS)
+@pytest.mark.parametrize("num_ctas", [40, 65])
+def test_combine_many_segments(kernel, num_ctas):
+    """One long unit cut into more than 32 segments: the combine folds its sweeps of 32
+    segments online (running maximum and rescaled sums)."""
+    inp = make_decode(1, 16, 16, 1, 128, 8192, seed=23, ctx_lens=[8192])
+    out, lse = run_decode(inp, kernel, num_ctas=num_ctas)
+    ro, rl = oracle_decode(inp)
+    assert_parity(out, ro, f"C={num_ctas} out")
+    assert_parity(lse, rl, f"C={num_ctas} lse")
+
+
 @pytest.fixture(scope="module")
 def wl2():
     return make_workload(2)
