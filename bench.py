@@ -360,6 +360,31 @@ def run_native(args):
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": round(ms_e2e, 4),
                "steps": n_e2e}
 
+    # ---- committed-block cache update at this workload's shape (decode only) ----
+    kv_app = None
+    if w.kind == "decode":
+        B_, S_, H_, D_ = w.batch, w.block_size, w.num_kv_heads, w.head_dim
+        aplan = ops.Plan(B_, w.num_q_heads, H_, D_, S_, ctx_capacity=2 * S_, device=local)
+        k_new = torch.empty((B_, S_, H_, D_), dtype=torch.bfloat16, device=dev).normal_()
+        v_new = torch.empty_like(k_new).normal_()
+        kc = torch.zeros((B_, H_, 2 * S_, D_), dtype=torch.bfloat16, device=dev)
+        vc = torch.zeros_like(kc)
+        zl = torch.zeros((B_,), dtype=torch.int32, device=dev)
+        for _ in range(3):
+            aplan.kv_append(k_new, v_new, kc, vc, zl, advance=False)
+        n_app = 50
+        b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        b0.record(stream)
+        for _ in range(n_app):
+            aplan.kv_append(k_new, v_new, kc, vc, zl, advance=False)
+        b1.record(stream)
+        torch.cuda.synchronize()
+        aplan.check()
+        us = b0.elapsed_time(b1) * 1e3 / n_app
+        nbytes = 4 * B_ * S_ * H_ * D_ * 2       # K and V: read the new rows, write them into the cache
+        kv_app = {"us_per_call": round(us, 3), "bytes": nbytes, "gbs": round(nbytes / (us * 1e-6) / 1e9, 2),
+                  "launches": n_app}
+
     # ---- oracle CPU baseline (rank 0, N = 1 only) ----
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
@@ -403,6 +428,7 @@ def run_native(args):
         "kernel": kname,
         "num_ctas": info.num_ctas,
         "e2e": e2e,
+        "kv_append": kv_app,
         "cpu_baseline": cpu,
         "clocks": ck,
     }

@@ -173,6 +173,23 @@ TT_API tt_status_t tt_block_attn_noalloc(const tt_block_attn_desc* desc, const v
                                          const int32_t* ctx_lens, float* out, float* lse, uint32_t* status,
                                          tt_stream_t stream);
 
+/* Committed-block cache update (paperfeed.app review of arXiv 2606.26493, section
+ * "The idea: freeze the reader, train the writer": a committed block is ingested by
+ * the frozen context tower, "updating its caches").  For every sequence n:
+ *   k_ctx[n, h, L_n + t, :] = k_new[n, t, h, :],  v_ctx likewise,  t < S, h < Hkv,
+ * with L_n = ctx_lens[n] read on the device, and then, when `advance` is non-zero,
+ * ctx_lens[n] = L_n + S.
+ *   k_new, v_new [B, S, Hkv, D] bf16  the context tower's layer-i K/V of the S committed
+ *                                     positions (computed by the caller)
+ *   k_ctx, v_ctx [B, Hkv, Lcap, D] bf16, updated in place; other rows are not touched
+ *   ctx_lens     [B] int32 on the device, read (and advanced) in place
+ * Uses the plan's B, S, Hkv, D and Lcap (ctx_capacity); asynchronous on `stream`.
+ * A sequence with L_n < 0 or L_n + S > Lcap is left untouched (rows and length) and
+ * raises TT_ERR_DEVICE_ARG at the next tt_block_attn_check.  Host-detectable errors
+ * (null or misaligned pointers, Lcap < S) return TT_ERR_INVALID_ARG. */
+TT_API tt_status_t tt_kv_append(tt_plan_t plan, const void* k_new, const void* v_new, void* k_ctx, void* v_ctx,
+                                int32_t* ctx_lens, int advance, tt_stream_t stream);
+
 /* Synchronise `stream`, then read and clear the plan's device error word.
  * Returns TT_OK, TT_ERR_DEVICE_ARG or TT_ERR_TIMEOUT (or TT_ERR_CUDA if the
  * synchronisation itself failed). */

@@ -276,3 +276,51 @@ def test_profile_hook_counts_launches(kernel):
     n, ms = plan.profile_read(0)
     plan.profile(False)
     assert n == 5 and ms > 0
+
+
+# --- committed-block cache update -------------------------------------------------
+def _bits(shape, rng):
+    """Random 16-bit patterns (every bf16 value, NaN and Inf patterns included)."""
+    return rng.integers(0, 1 << 16, size=shape, dtype=np.uint16)
+
+
+def _dev_bits(a):
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda()
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("advance", [True, False])
+def test_kv_append_bit_exact(D, advance):
+    from oracle import kv_append as oracle_append
+    rng = np.random.default_rng(31 + D)
+    B, S, Hkv, Lcap = 4, 16, 2, 100
+    lens = np.array([0, 50, 84, 85], dtype=np.int32)          # the last has no room
+    k_new, v_new = _bits((B, S, Hkv, D), rng), _bits((B, S, Hkv, D), rng)
+    k_ctx, v_ctx = _bits((B, Hkv, Lcap, D), rng), _bits((B, Hkv, Lcap, D), rng)
+    plan = ops.Plan(B, 4, Hkv, D, S, ctx_capacity=Lcap)
+    dk, dv, dl = _dev_bits(k_ctx), _dev_bits(v_ctx), torch.from_numpy(lens).cuda()
+    plan.kv_append(_dev_bits(k_new), _dev_bits(v_new), dk, dv, dl, advance=advance)
+    assert plan.check_status() == ops.TT_ERR_DEVICE_ARG         # sequence 3 was reported
+    rk, rv, rl, bad = oracle_append(k_new, v_new, k_ctx, v_ctx, lens, advance=advance)
+    assert list(bad) == [False, False, False, True]
+    assert np.array_equal(dk.cpu().numpy().view(np.uint16), rk)
+    assert np.array_equal(dv.cpu().numpy().view(np.uint16), rv)
+    assert np.array_equal(dl.cpu().numpy(), rl.astype(np.int32))
+
+
+def test_kv_append_then_decode_equals_decode_with_block_in_context():
+    """Commit block b (its context-tower K/V) and decode the next block: the same as
+    decoding that block with the committed rows already in the cache."""
+    from oracle import kv_append as oracle_append
+    inp = make_decode(2, 16, 32, 2, 128, 600, seed=33, ctx_lens=[300, 584])
+    k_new = make_decode(2, 16, 32, 2, 128, 1, seed=35).k_blk      # bf16 bits [B, S, Hkv, D]
+    v_new = make_decode(2, 16, 32, 2, 128, 1, seed=36).v_blk
+    plan = ops.Plan(2, 32, 2, 128, 16, ctx_capacity=600)
+    dk, dv, dl = dev(inp.k_ctx).clone(), dev(inp.v_ctx).clone(), torch.from_numpy(inp.ctx_lens).cuda()
+    plan.kv_append(dev(k_new), dev(v_new), dk, dv, dl)
+    out, lse = plan.block_attn(dev(inp.q), dk, dv, dev(inp.k_blk), dev(inp.v_blk), dl, want_lse=True)
+    plan.check()
+    rk, rv, rl, _ = oracle_append(k_new, v_new, inp.k_ctx, inp.v_ctx, inp.ctx_lens)
+    ro, rlse = oracle_attn(f64(inp.q), f64(rk), f64(rv), f64(inp.k_blk), f64(inp.v_blk), rl)
+    assert_parity(out, ro, "out after append")
+    assert_parity(lse, rlse, "lse after append")

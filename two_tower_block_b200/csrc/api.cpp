@@ -14,6 +14,7 @@
 
 #include "../../include/tt_block_attn.h"
 #include "problem.h"
+#include "kv_append.h"
 #include "errbits.h"
 #include "sched.cuh"
 
@@ -474,6 +475,24 @@ tt_status_t tt_block_attn_host(tt_plan_t plan, const void* q, const void* k_ctx,
   return TT_OK;
 }
 
+tt_status_t tt_kv_append(tt_plan_t plan, const void* k_new, const void* v_new, void* k_ctx, void* v_ctx,
+                         int32_t* ctx_lens, int advance, tt_stream_t stream) {
+  if (!plan) return fail(TT_ERR_INVALID_ARG, "null plan");
+  const tt_block_attn_desc& d = plan->desc;
+  if (d.batch == 0) return TT_OK;
+  if (d.ctx_capacity < d.block_size) return fail(TT_ERR_INVALID_ARG, "plan's ctx_capacity has no room for a block");
+  if (!k_new || !v_new || !k_ctx || !v_ctx || !ctx_lens) return fail(TT_ERR_INVALID_ARG, "null tensor pointer");
+  if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_ctx) || !aligned16(v_ctx) ||
+      (reinterpret_cast<uintptr_t>(ctx_lens) & 3u))
+    return fail(TT_ERR_INVALID_ARG, "tensor pointer not 16-byte aligned");
+  DeviceGuard guard(plan->device);
+  cudaError_t e = tt::launch_kv_append(k_new, v_new, k_ctx, v_ctx, ctx_lens, d.batch, d.block_size, d.num_kv_heads,
+                                       d.head_dim, d.ctx_capacity, advance ? 1 : 0, plan->err_word,
+                                       reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "kv_append launch");
+  return TT_OK;
+}
+
 tt_status_t tt_block_attn_check(tt_plan_t plan, tt_stream_t stream) {
   if (!plan) return fail(TT_ERR_INVALID_ARG, "null plan");
   DeviceGuard guard(plan->device);
@@ -486,7 +505,9 @@ tt_status_t tt_block_attn_check(tt_plan_t plan, tt_stream_t stream) {
   if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
   if (w & tt::kErrInternal) return fail(TT_ERR_CUDA, "a kernel found its launch unusable (internal error)");
   if (w & tt::kErrTimeout) return fail(TT_ERR_TIMEOUT, "an in-kernel wait timed out");
-  if (w & tt::kErrDeviceArg) return fail(TT_ERR_DEVICE_ARG, "ctx_lens value outside [0, ctx_capacity]");
+  if (w & tt::kErrDeviceArg)
+    return fail(TT_ERR_DEVICE_ARG,
+                "ctx_lens value out of range (attention: [0, ctx_capacity]; kv append: [0, ctx_capacity - block])");
   return TT_OK;
 }
 

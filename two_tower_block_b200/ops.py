@@ -31,7 +31,7 @@ EXPORTED_SYMBOLS = [
     "tt_block_attn_plan", "tt_block_attn_plan_destroy", "tt_block_attn_plan_get_info", "tt_block_attn",
     "tt_block_attn_block_causal", "tt_block_attn_host", "tt_block_attn_check", "tt_block_attn_profile",
     "tt_block_attn_profile_read", "tt_selftest_wait_timeout", "tt_debug_work_split", "tt_status_string",
-    "tt_last_error_detail", "tt_block_attn_noalloc", "tt_selftest_exp2",
+    "tt_last_error_detail", "tt_block_attn_noalloc", "tt_selftest_exp2", "tt_kv_append",
 ]
 
 
@@ -190,6 +190,13 @@ class Plan:
                                                 _ptr(v_blk), _ptr(out), _ptr(lse), _stream(stream)),
                "tt_block_attn_block_causal")
         return (out, lse) if want_lse or lse is not None else out
+
+    # --- committed-block cache update ------------------------------------------
+    def kv_append(self, k_new, v_new, k_ctx, v_ctx, ctx_lens, advance=True, stream=None):
+        """Write k_new/v_new [B,S,Hkv,D] into k_ctx/v_ctx [B,Hkv,Lcap,D] at [L_n, L_n+S) in
+        place; advance ctx_lens (device int32) by S when `advance`."""
+        _check(lib().tt_kv_append(self._h, _ptr(k_new), _ptr(v_new), _ptr(k_ctx), _ptr(v_ctx), _ptr(ctx_lens),
+                                  int(bool(advance)), _stream(stream)), "tt_kv_append")
 
     # --- status / timing ---------------------------------------------------
     def check(self, stream=None):
