@@ -328,7 +328,8 @@ def run_native(args):
     plan.check()
     ms_total = max_over_ranks(pg, ms_total, dev)
     ms_step = ms_total / args.steps
-    launches_per_step = 1 + (1 if info.num_ctas > 1 else 0)
+    # one attention launch per step, plus the split combine when it ran as its own kernel
+    launches_per_step = 1 + (1 if n_c > 0 else 0)
 
     # ---- end to end through the host-buffer entry (decode workloads) ----
     e2e = None

@@ -93,6 +93,8 @@ struct tt_plan_s {
   float* part_lse = nullptr;
   tt::SplitRecord* records = nullptr;
   unsigned* err_word = nullptr;
+  unsigned long long* grid_bar = nullptr;  // fused combine's grid barrier (in the error-word block)
+  bool fused_combine = false;
   int* causal_pref = nullptr;
   long long causal_T = 0;
   int causal_NB = 0;
@@ -154,6 +156,7 @@ tt::Problem base_problem(tt_plan_t plan) {
   p.err_word = plan->err_word;
   p.wait_limit_ns = (unsigned long long)(d.wait_timeout_us > 0 ? d.wait_timeout_us : 1000000) * 1000ull;
   p.variant = plan->variant;
+  p.grid_bar = plan->fused_combine ? plan->grid_bar : nullptr;
   return p;
 }
 
@@ -201,7 +204,7 @@ tt_status_t launch_all(tt_plan_t plan, const tt::Problem& p, cudaStream_t s) {
   }
   prof_mark(plan, 0, s, false);
   if (e != cudaSuccess) return cuda_fail(e, "attention kernel launch");
-  if (plan->C > 1) {
+  if (plan->C > 1 && p.grid_bar == nullptr) {
     prof_mark(plan, 1, s, true);
     e = tt::launch_combine(p, s);
     prof_mark(plan, 1, s, false);
@@ -329,6 +332,16 @@ tt_status_t tt_block_attn_plan(const tt_block_attn_desc* desc, int device, tt_pl
   P->part_lse = reinterpret_cast<float*>(w + b_po);
   P->records = reinterpret_cast<tt::SplitRecord*>(w + b_po + b_pl);
   P->err_word = reinterpret_cast<unsigned*>(w + b_po + b_pl + b_rec);
+  P->grid_bar = reinterpret_cast<unsigned long long*>(w + b_po + b_pl + b_rec + 128);
+  // TT_FUSED_COMBINE=1: the default tcgen05 kernel combines the cut units itself when all
+  // its CTAs can be resident at once (one per SM): a cooperative launch with a grid
+  // barrier at the end.  Off by default: waiting for the slowest CTA costs more than the
+  // separate combine kernel's launch.
+  {
+    const char* fc = std::getenv("TT_FUSED_COMBINE");
+    P->fused_combine = P->kernel == TT_KERNEL_TCGEN05 && P->variant == 0 && P->C > 1 && P->C <= P->sm_count &&
+                       fc && std::atoi(fc) == 1;
+  }
   P->causal_pref = pref.empty() ? nullptr : reinterpret_cast<int*>(w + b_po + b_pl + b_rec + b_err);
   e = cudaMemset(P->err_word, 0, b_err);
   if (e == cudaSuccess && !pref.empty())

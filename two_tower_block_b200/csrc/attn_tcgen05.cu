@@ -34,6 +34,7 @@
 //
 // Every wait is bounded (ptx.cuh: mbar_wait); on a timeout the CTA raises the
 // error word, drains what it issued, frees TMEM and returns.
+#include "combine_row.cuh"
 #include "problem.h"
 #include "ptx.cuh"
 #include "tc_common.cuh"
@@ -80,6 +81,62 @@ struct Shared {
   long long T, start, end;
   Unit first;
 };
+
+// Fused split combine (cooperative launch only): every CTA arrives at a grid barrier once
+// its segments and its split record are written, then the CTAs share the rows of the cut
+// units, one warp per row.  `scratch` holds C records and C indices.  The wait is bounded;
+// a CTA that gave up (or whose pipeline aborted) combines nothing and the error word says so.
+template <int D>
+__device__ __forceinline__ void fused_combine(const Problem& p, uint8_t* scratch, bool aborted) {
+  __shared__ int s_go, s_ncut;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  __syncthreads();  // every write of this CTA precedes its arrival
+  if (tid == 0) {
+    __threadfence();
+    const unsigned long long old = atomicAdd(p.grid_bar, 1ull);
+    const unsigned long long target = (old / (unsigned long long)p.C + 1ull) * (unsigned long long)p.C;
+    const unsigned long long t0 = globaltimer_ns();
+    bool ok = true;
+    while (ld_acquire_gpu(p.grid_bar) < target) {
+      if (globaltimer_ns() - t0 > p.wait_limit_ns) {
+        raise_error(p.err_word, kErrTimeout);
+        ok = false;
+        break;
+      }
+      __nanosleep(64);
+    }
+    __threadfence();
+    s_go = ok && !aborted;
+  }
+  __syncthreads();
+  if (!s_go) return;
+  SplitRecord* recs = reinterpret_cast<SplitRecord*>(scratch);
+  int* cut = reinterpret_cast<int*>(scratch + p.C * sizeof(SplitRecord));
+  for (int i = tid; i < p.C; i += kThreads) {
+    const int4 v = __ldcg(reinterpret_cast<const int4*>(p.records + i));
+    recs[i] = SplitRecord{v.x, v.y, v.z, v.w};
+  }
+  __syncthreads();
+  if (warp == 0) {
+    int n = 0;
+    for (int base = 0; base < p.C; base += 32) {
+      const int i = base + lane;
+      const bool is_cut = i < p.C && recs[i].unit >= 0;
+      const unsigned m = __ballot_sync(0xffffffffu, is_cut);
+      if (is_cut) cut[n + __popc(m & ((1u << lane) - 1u))] = i;
+      n += __popc(m);
+    }
+    if (lane == 0) s_ncut = n;
+  }
+  __syncthreads();
+  const int nw = kThreads / 32;
+  const long long jobs = (long long)s_ncut * p.R;
+  for (long long job = (long long)blockIdx.x * nw + warp; job < jobs; job += (long long)p.C * nw) {
+    const int k = (int)(job / p.R), r = (int)(job - (long long)k * p.R);
+    const int c = cut[k];
+    combine_row<D>(p, c, recs[c], r, lane);
+  }
+}
 
 template <int D, int NK>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -458,6 +515,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem, 512);
+  if (p.grid_bar != nullptr) fused_combine<D>(p, smem + C::kEpiOff, *(volatile int*)&sh->abort_flag != 0);
 }
 
 template <int D, int NK>
@@ -467,8 +525,23 @@ void set_smem_attr() {
 }
 
 template <int D, int NK>
-void launch(const Problem& p, const TmaMaps& maps, cudaStream_t stream) {
-  attn_tcgen05_kernel<D, NK><<<p.C, kThreads, Cfg<D, NK>::kSmemBytes, stream>>>(p, maps);
+cudaError_t launch(const Problem& p, const TmaMaps& maps, cudaStream_t stream) {
+  if (p.grid_bar == nullptr) {
+    attn_tcgen05_kernel<D, NK><<<p.C, kThreads, Cfg<D, NK>::kSmemBytes, stream>>>(p, maps);
+    return cudaGetLastError();
+  }
+  // cooperative: every CTA must be resident at once for the grid barrier of the fused combine
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.C, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = Cfg<D, NK>::kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, attn_tcgen05_kernel<D, NK>, p, maps);
 }
 
 }  // namespace
@@ -487,14 +560,8 @@ cudaError_t launch_attn_tcgen05(const Problem& p, const TmaMaps& maps, cudaStrea
   if (!tcgen05_key_tile_supported(p.key_tile)) return cudaErrorInvalidValue;
   // variant 2: head_dim 128 with 128-key tiles on the transposed-PV kernel (attn_tcgen05_pt.cu)
   if (p.D == 128 && p.key_tile == 128 && p.variant == 2) return launch_attn_pt(p, maps, stream);
-  if (p.D == 128) {
-    if (p.key_tile == 128) launch<128, 128>(p, maps, stream);
-    else launch<128, 64>(p, maps, stream);
-  } else {
-    if (p.key_tile == 128) launch<64, 128>(p, maps, stream);
-    else launch<64, 64>(p, maps, stream);
-  }
-  return cudaGetLastError();
+  if (p.D == 128) return p.key_tile == 128 ? launch<128, 128>(p, maps, stream) : launch<128, 64>(p, maps, stream);
+  return p.key_tile == 128 ? launch<64, 128>(p, maps, stream) : launch<64, 64>(p, maps, stream);
 }
 
 }  // namespace tt

@@ -47,6 +47,10 @@ struct Problem {
   unsigned long long wait_limit_ns;
   int variant;          // tcgen05 kernel: 0 = S/P aliasing in TMEM (default), 2 = transposed PV,
                         // 3 = 2-SM pairs (head_dim 128)
+  // default tcgen05 kernel launched cooperatively: the CTAs meet at this grid barrier
+  // (a counter that only grows) and combine the cut units themselves; null: the
+  // separate combine kernel runs instead
+  unsigned long long* grid_bar;
 };
 
 // Host launchers (each returns the cudaError_t of its launch).
