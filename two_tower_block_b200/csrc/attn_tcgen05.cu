@@ -158,10 +158,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // ---------------------------------------------------------------- setup --
   {
-    // zero Q (rows >= R stay zero for every segment) through the generic proxy
-    uint4* z = reinterpret_cast<uint4*>(smem);
-    for (int i = tid; i < C::kQBytes / 16; i += kThreads) z[i] = make_uint4(0, 0, 0, 0);
-    fence_proxy_async_smem();
+    // zero Q (rows >= R stay zero for every segment) through the generic proxy; when R
+    // fills its M-tiles every row is loaded by TMA and nothing needs clearing
+    if (p.R % 128 != 0) {
+      uint4* z = reinterpret_cast<uint4*>(smem);
+      for (int i = tid; i < C::kQBytes / 16; i += kThreads) z[i] = make_uint4(0, 0, 0, 0);
+      fence_proxy_async_smem();
+    }
   }
   if (tid == 0) {
     mbar_init(smem_u32(&bars->q_full), 1);
