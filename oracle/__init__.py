@@ -6,3 +6,4 @@ Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline legs of
 from .oracle import attend_rows, block_attn, block_causal  # noqa: F401
 from .brute import brute_block_attn, brute_block_causal  # noqa: F401
 from .kv_append import kv_append  # noqa: F401
+from .backward import block_causal_backward  # noqa: F401
