@@ -361,6 +361,39 @@ def run_native(args):
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": round(ms_e2e, 4),
                "steps": n_e2e}
 
+    # ---- block-causal backward at this workload's shape (training workloads) ----
+    bwd = None
+    if w.kind == "causal":
+        c0 = copies[0]
+        bout = torch.empty((w.batch, w.seq_len, w.num_q_heads, w.head_dim), dtype=torch.float32, device=dev)
+        blse = torch.empty((w.batch, w.num_q_heads, w.seq_len), dtype=torch.float32, device=dev)
+        plan.block_attn_block_causal(c0[0], c0[1], c0[2], c0[3], c0[4], out=bout, lse=blse)
+        dout = torch.empty_like(bout).normal_().to(torch.bfloat16)
+        dq = torch.empty_like(bout)
+        dkb = torch.empty((w.batch, w.seq_len, w.num_kv_heads, w.head_dim), dtype=torch.float32, device=dev)
+        dvb = torch.empty_like(dkb)
+        for _ in range(2):
+            plan.block_causal_backward(c0[0], c0[1], c0[2], c0[3], c0[4], bout, blse, dout, dq, dkb, dvb)
+        torch.cuda.synchronize()
+        plan.profile(True)
+        n_b = 3
+        for _ in range(n_b):
+            plan.block_causal_backward(c0[0], c0[1], c0[2], c0[3], c0[4], bout, blse, dout, dq, dkb, dvb)
+        torch.cuda.synchronize()
+        nb_l, ms_b = plan.profile_read(2)
+        plan.profile(False)
+        plan.check()
+        ms_b /= max(nb_l, 1)
+        # recompute S, dP and dQ over every visible key (3 x 2D flops per row and key),
+        # dK and dV over the block's own keys (2 x 2D per row and block key)
+        rows_keys = cost["flops"] / (4 * w.head_dim)
+        rows_blk = w.batch * w.num_q_heads * w.seq_len * w.block_size
+        bflops = 6 * w.head_dim * rows_keys + 4 * w.head_dim * rows_blk
+        pkk = load_peaks()
+        pk = pkk["bf16_tflops_sustained"] or pkk["bf16_tflops"]
+        bwd = {"kernel": "attn_bwd (mma.sync)", "ms": round(ms_b, 4), "tflops": round(bflops / (ms_b * 1e-3) / 1e12, 2),
+               "frac_of_sustained_bf16": round(bflops / (ms_b * 1e-3) / 1e12 / pk, 4), "launches": nb_l}
+
     # ---- committed-block cache update at this workload's shape (decode only) ----
     kv_app = None
     if w.kind == "decode":
@@ -436,6 +469,7 @@ def run_native(args):
         "num_ctas": info.num_ctas,
         "e2e": e2e,
         "kv_append": kv_app,
+        "backward": bwd,
         "cpu_baseline": cpu,
         "clocks": ck,
     }

@@ -173,6 +173,27 @@ TT_API tt_status_t tt_block_attn_noalloc(const tt_block_attn_desc* desc, const v
                                          const int32_t* ctx_lens, float* out, float* lse, uint32_t* status,
                                          tt_stream_t stream);
 
+/* Block-causal backward pass (paperfeed.app review of arXiv 2606.26493, section
+ * "Training and sampling": the loss of block b is conditioned on the noisy block and
+ * the frozen caches c_{<b}; the context tower runs without gradients).  Gradients of
+ * sum(dout * out) with respect to the denoiser's queries and its own block keys and
+ * values; the context cache gets none.  For the rows r of block b and the keys k of
+ * its key set (context positions < S*b, then its own S positions):
+ *   p = exp(scale q.k - lse),  ds = p (dout.v - dout.out),
+ *   dq = scale sum_k ds k,  dk_blk[k] = scale sum_r ds q_r,  dv_blk[k] = sum_r p dout_r
+ * (block keys only; summed over the g query heads of each KV head).
+ *   q, k_ctx, v_ctx, k_blk, v_blk   the forward's inputs, layouts of tt_block_attn_block_causal
+ *   out  [B, N, Hq, D] fp32, lse [B, Hq, N] fp32   the forward's outputs (lse required)
+ *   dout [B, N, Hq, D] bf16        dL/dout (a bf16 operand of the tensor cores, like q, k, v)
+ *   dq   [B, N, Hq, D] fp32        written
+ *   dk_blk, dv_blk [B, N, Hkv, D] fp32   cleared, then written
+ * The plan must be a block-causal plan (seq_len > 0).  Asynchronous on `stream`. */
+TT_API tt_status_t tt_block_attn_block_causal_backward(tt_plan_t plan, const void* q, const void* k_ctx,
+                                                       const void* v_ctx, const void* k_blk, const void* v_blk,
+                                                       const float* out, const float* lse, const void* dout,
+                                                       float* dq, float* dk_blk, float* dv_blk,
+                                                       tt_stream_t stream);
+
 /* Committed-block cache update (paperfeed.app review of arXiv 2606.26493, section
  * "The idea: freeze the reader, train the writer": a committed block is ingested by
  * the frozen context tower, "updating its caches").  For every sequence n:
@@ -198,8 +219,9 @@ TT_API tt_status_t tt_block_attn_check(tt_plan_t plan, tt_stream_t stream);
 /* Per-kernel timing hook.  While enabled, every kernel the plan launches is
  * bracketed by two CUDA events recorded on the launching stream (up to 4096
  * launches are kept).  tt_block_attn_profile_read synchronises on the recorded
- * events and returns, for kernel id 0 (attention) or 1 (split combine), the
- * number of launches and their summed duration in milliseconds.  Calling
+ * events and returns, for kernel id 0 (attention), 1 (split combine) or 2
+ * (block-causal backward), the number of launches and their summed duration in
+ * milliseconds.  Calling
  * tt_block_attn_profile again clears the record. */
 TT_API tt_status_t tt_block_attn_profile(tt_plan_t plan, int enable);
 TT_API tt_status_t tt_block_attn_profile_read(tt_plan_t plan, int kernel_id, int* launches, double* total_ms);

@@ -12,9 +12,9 @@ import torch
 
 from oracle import block_attn as oracle_attn
 from oracle import block_causal as oracle_causal
-from tests.gpu_util import assert_parity, dev, f64, poison_beyond
+from tests.gpu_util import assert_parity, dev, errors, f64, poison_beyond
 from two_tower_block_b200 import ops
-from two_tower_block_b200.workloads import WORKLOADS, make_causal, make_decode, make_workload
+from two_tower_block_b200.workloads import WORKLOADS, bf16_bits, make_causal, make_decode, make_workload
 
 pytestmark = pytest.mark.gpu
 
@@ -326,3 +326,54 @@ def test_kv_append_then_decode_equals_decode_with_block_in_context():
     ro, rlse = oracle_attn(f64(inp.q), f64(rk), f64(rv), f64(inp.k_blk), f64(inp.v_blk), rl)
     assert_parity(out, ro, "out after append")
     assert_parity(lse, rlse, "lse after append")
+
+
+# --- block-causal backward ------------------------------------------------------------
+def run_backward(inp, dout_bits, kernel=(ops.KERNEL_TCGEN05, {})):
+    B, N, Hq, D = inp.q.shape
+    Hkv = inp.k_ctx.shape[1]
+    plan = make_plan(kernel, B, Hq, Hkv, D, inp.block_size, seq_len=N)
+    q, kc, vc, kb, vb = dev(inp.q), dev(inp.k_ctx), dev(inp.v_ctx), dev(inp.k_blk), dev(inp.v_blk)
+    out, lse = plan.block_attn_block_causal(q, kc, vc, kb, vb, want_lse=True)
+    dq, dk, dv = plan.block_causal_backward(q, kc, vc, kb, vb, out, lse, dev(dout_bits))
+    plan.check()
+    return dq, dk, dv
+
+
+@pytest.mark.parametrize("shape", [(2, 64, 16, 8, 2, 128), (1, 40, 4, 8, 1, 64), (2, 300, 20, 4, 2, 128),
+                                   (1, 256, 128, 2, 1, 64)],
+                         ids=["S16-g4-D128", "S4-g8-D64", "S20-g2-D128-ragged", "S128-g2-D64"])
+def test_block_causal_backward_small(shape):
+    from oracle import block_causal_backward
+    B, N, S, Hq, Hkv, D = shape
+    inp = make_causal(B, N, S, Hq, Hkv, D, seed=41)
+    dout = bf16_bits(np.random.default_rng(42).standard_normal((B, N, Hq, D)).astype(np.float32))
+    dq, dk, dv = run_backward(inp, dout)
+    rq, rk, rv = block_causal_backward(f64(inp.q), f64(inp.k_ctx), f64(inp.v_ctx), f64(inp.k_blk),
+                                       f64(inp.v_blk), f64(dout), S)
+    errs = {w: errors(a, r) for w, a, r in (("dq", dq, rq), ("dk_blk", dk, rk), ("dv_blk", dv, rv))}
+    print({w: (f"{e[0]:.2e}", f"{e[1]:.2e}") for w, e in errs.items()})
+    assert_parity(dq, rq, "dq")
+    assert_parity(dk, rk, "dk_blk")
+    assert_parity(dv, rv, "dv_blk")
+
+
+def test_block_causal_backward_full_sampled():
+    """The full N=8192 training workload on the GPU; oracle on a few blocks spread over
+    the sequence (early, middle, last) of sequence 0."""
+    from oracle import block_causal_backward
+    inp = make_workload(5)
+    B, N, Hq, D = inp.q.shape
+    S = inp.block_size
+    dout = bf16_bits(np.random.default_rng(43).standard_normal((B, N, Hq, D)).astype(np.float32))
+    dq, dk, dv = run_backward(inp, dout)
+    assert torch.isfinite(dq).all() and torch.isfinite(dk).all() and torch.isfinite(dv).all()
+    blocks = [0, 1, 255, 511]
+    rq, rk, rv = block_causal_backward(f64(inp.q[:1]), f64(inp.k_ctx[:1]), f64(inp.v_ctx[:1]),
+                                       f64(inp.k_blk[:1]), f64(inp.v_blk[:1]), f64(dout[:1]), S,
+                                       blocks=blocks)
+    for b in blocks:
+        sl = slice(S * b, S * b + S)
+        assert_parity(dq[:1, sl], rq[:, sl], f"dq block {b}")
+        assert_parity(dk[:1, sl], rk[:, sl], f"dk_blk block {b}")
+        assert_parity(dv[:1, sl], rv[:, sl], f"dv_blk block {b}")

@@ -15,6 +15,7 @@
 #include "../../include/tt_block_attn.h"
 #include "problem.h"
 #include "kv_append.h"
+#include "attn_bwd.h"
 #include "errbits.h"
 #include "sched.cuh"
 
@@ -485,6 +486,56 @@ tt_status_t tt_block_attn_host(tt_plan_t plan, const void* q, const void* k_ctx,
   e = cudaMemcpyAsync(out, dout, B * S * Hq * D * 4, cudaMemcpyDeviceToHost, s);
   if (e == cudaSuccess && lse) e = cudaMemcpyAsync(lse, dlse, B * Hq * S * 4, cudaMemcpyDeviceToHost, s);
   if (e != cudaSuccess) return cuda_fail(e, "device-to-host copy");
+  return TT_OK;
+}
+
+tt_status_t tt_block_attn_block_causal_backward(tt_plan_t plan, const void* q, const void* k_ctx, const void* v_ctx,
+                                                const void* k_blk, const void* v_blk, const float* out,
+                                                const float* lse, const void* dout, float* dq, float* dk_blk,
+                                                float* dv_blk, tt_stream_t stream) {
+  if (!plan) return fail(TT_ERR_INVALID_ARG, "null plan");
+  const tt_block_attn_desc& d = plan->desc;
+  if (d.seq_len == 0) return fail(TT_ERR_INVALID_ARG, "plan has seq_len == 0 (decode-only)");
+  if (d.batch == 0) return TT_OK;
+  if (!q || !k_ctx || !v_ctx || !k_blk || !v_blk || !out || !lse || !dout || !dq || !dk_blk || !dv_blk)
+    return fail(TT_ERR_INVALID_ARG, "null tensor pointer");
+  if (!aligned16(q) || !aligned16(k_ctx) || !aligned16(v_ctx) || !aligned16(k_blk) || !aligned16(v_blk) ||
+      !aligned16(out) || !aligned16(dout) || !aligned16(dq) || !aligned16(dk_blk) || !aligned16(dv_blk) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return fail(TT_ERR_INVALID_ARG, "tensor pointer not 16-byte aligned");
+  DeviceGuard guard(plan->device);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  tt::BwdProblem p{};
+  p.B = d.batch;
+  p.Hq = d.num_q_heads;
+  p.Hkv = d.num_kv_heads;
+  p.g = plan->g;
+  p.D = d.head_dim;
+  p.S = d.block_size;
+  p.R = plan->R;
+  p.N = d.seq_len;
+  p.NB = d.seq_len / d.block_size;
+  p.scale = plan->scale;
+  p.scale_log2 = plan->scale * 1.4426950408889634f;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.k_ctx = static_cast<const __nv_bfloat16*>(k_ctx);
+  p.v_ctx = static_cast<const __nv_bfloat16*>(v_ctx);
+  p.k_blk = static_cast<const __nv_bfloat16*>(k_blk);
+  p.v_blk = static_cast<const __nv_bfloat16*>(v_blk);
+  p.out = out;
+  p.lse = lse;
+  p.dout = static_cast<const __nv_bfloat16*>(dout);
+  p.dq = dq;
+  p.dk_blk = dk_blk;
+  p.dv_blk = dv_blk;
+  const size_t kv_bytes = (size_t)d.batch * d.seq_len * d.num_kv_heads * d.head_dim * sizeof(float);
+  cudaError_t e = cudaMemsetAsync(dk_blk, 0, kv_bytes, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(dv_blk, 0, kv_bytes, s);
+  if (e != cudaSuccess) return cuda_fail(e, "clearing dk_blk / dv_blk");
+  prof_mark(plan, 2, s, true);
+  e = tt::launch_attn_bwd(p, s);
+  prof_mark(plan, 2, s, false);
+  if (e != cudaSuccess) return cuda_fail(e, "backward kernel launch");
   return TT_OK;
 }
 

@@ -32,6 +32,7 @@ EXPORTED_SYMBOLS = [
     "tt_block_attn_block_causal", "tt_block_attn_host", "tt_block_attn_check", "tt_block_attn_profile",
     "tt_block_attn_profile_read", "tt_selftest_wait_timeout", "tt_debug_work_split", "tt_status_string",
     "tt_last_error_detail", "tt_block_attn_noalloc", "tt_selftest_exp2", "tt_kv_append",
+    "tt_block_attn_block_causal_backward",
 ]
 
 
@@ -190,6 +191,23 @@ class Plan:
                                                 _ptr(v_blk), _ptr(out), _ptr(lse), _stream(stream)),
                "tt_block_attn_block_causal")
         return (out, lse) if want_lse or lse is not None else out
+
+    def block_causal_backward(self, q, k_ctx, v_ctx, k_blk, v_blk, out, lse, dout, dq=None, dk_blk=None,
+                              dv_blk=None, stream=None):
+        """Gradients (dq, dk_blk, dv_blk) of sum(dout * out) for the block-causal attention;
+        out and lse are the forward's outputs (fp32), dout is bf16."""
+        s = self.shape
+        if dq is None:
+            dq = torch.empty((s.batch, s.seq_len, s.q_heads, s.head_dim), dtype=torch.float32, device=q.device)
+        if dk_blk is None:
+            dk_blk = torch.empty((s.batch, s.seq_len, s.kv_heads, s.head_dim), dtype=torch.float32,
+                                 device=q.device)
+        if dv_blk is None:
+            dv_blk = torch.empty_like(dk_blk)
+        _check(lib().tt_block_attn_block_causal_backward(
+            self._h, _ptr(q), _ptr(k_ctx), _ptr(v_ctx), _ptr(k_blk), _ptr(v_blk), _ptr(out), _ptr(lse), _ptr(dout),
+            _ptr(dq), _ptr(dk_blk), _ptr(dv_blk), _stream(stream)), "tt_block_attn_block_causal_backward")
+        return dq, dk_blk, dv_blk
 
     # --- committed-block cache update ------------------------------------------
     def kv_append(self, k_new, v_new, k_ctx, v_ctx, ctx_lens, advance=True, stream=None):
