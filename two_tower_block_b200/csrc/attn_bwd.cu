@@ -15,7 +15,9 @@
 // dP = dO V^T, dS, dQ += dS K (dQ stays in registers for the whole key list).  On the
 // block's own tiles, P and dS go through shared memory and every warp forms
 // dK = dS^T Q and dV = P^T dO for 16 of the keys, added with fp32 atomics (the CTAs
-// of a unit's row chunks and the g query heads of a KV head all contribute).
+// of a unit's row chunks and the g query heads of a KV head all contribute).  dS and
+// P enter these products as bf16 pairs hi + lo, so the gradients carry only the
+// rounding of the bf16 inputs.
 #include "attn_bwd.h"
 
 #include "errbits.h"
@@ -175,14 +177,19 @@ __global__ void __launch_bounds__(kThreads) attn_bwd_kernel(const BwdProblem p) 
       dp[nb][2] = p2 * (dp[nb][2] - del_b);
       dp[nb][3] = p3 * (dp[nb][3] - del_b);
     }
-    // ---- dQ += dS K  (A = dS from registers, B = K rows via transposed loads) ----
+    // ---- dQ += dS K  (A = dS from registers as a bf16 pair hi + lo, B = K rows via
+    //      transposed loads): dq does not inherit a bf16 rounding of dS ----
+    auto split = [](float x0, float x1, uint32_t& hi, uint32_t& lo) {
+      hi = pack_bf16(x0, x1);
+      lo = pack_bf16(x0 - __uint_as_float(hi << 16), x1 - __uint_as_float(hi & 0xFFFF0000u));
+    };
 #pragma unroll
     for (int kk = 0; kk < kKeys / 16; ++kk) {
-      uint32_t pa[4];
-      pa[0] = pack_bf16(dp[2 * kk][0], dp[2 * kk][1]);
-      pa[1] = pack_bf16(dp[2 * kk][2], dp[2 * kk][3]);
-      pa[2] = pack_bf16(dp[2 * kk + 1][0], dp[2 * kk + 1][1]);
-      pa[3] = pack_bf16(dp[2 * kk + 1][2], dp[2 * kk + 1][3]);
+      uint32_t pa[4], pl[4];
+      split(dp[2 * kk][0], dp[2 * kk][1], pa[0], pl[0]);
+      split(dp[2 * kk][2], dp[2 * kk][3], pa[1], pl[1]);
+      split(dp[2 * kk + 1][0], dp[2 * kk + 1][1], pa[2], pl[2]);
+      split(dp[2 * kk + 1][2], dp[2 * kk + 1][3], pa[3], pl[3]);
 #pragma unroll
       for (int db2 = 0; db2 < D / 16; ++db2) {
         uint32_t b0, b1, b2, b3;
@@ -191,6 +198,8 @@ __global__ void __launch_bounds__(kThreads) attn_bwd_kernel(const BwdProblem p) 
         ldmatrix_x4_trans(a, b0, b1, b2, b3);
         mma_bf16_16816(dq[2 * db2], pa, b0, b1);
         mma_bf16_16816(dq[2 * db2 + 1], pa, b2, b3);
+        mma_bf16_16816(dq[2 * db2], pl, b0, b1);
+        mma_bf16_16816(dq[2 * db2 + 1], pl, b2, b3);
       }
     }
 
