@@ -425,6 +425,33 @@ def run_native(args):
         kv_app = {"us_per_call": round(us, 3), "bytes": nbytes, "gbs": round(nbytes / (us * 1e-6) / 1e9, 2),
                   "launches": n_app}
 
+    # ---- confidence-unmasking step over a 131072-entry vocabulary at the block shape ----
+    unmask = None
+    if w.kind == "decode":
+        Vv = 131072
+        lg = torch.empty((w.batch, w.block_size, Vv), dtype=torch.bfloat16, device=dev).normal_()
+        tk = torch.full((w.batch, w.block_size), -1, dtype=torch.int32, device=dev)
+        mk = torch.ones((w.batch, w.block_size), dtype=torch.uint8, device=dev)
+        # standard-normal logits never reach 0.8 and min_one is off: every call scans every row
+        for _ in range(3):
+            ops.confidence_unmask(lg, tk, mk, gamma=0.8, min_one=False)
+        ug = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(ug):
+            ops.confidence_unmask(lg, tk, mk, gamma=0.8, min_one=False)
+        ug.replay()
+        torch.cuda.synchronize()
+        u0, u1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n_u = 50
+        u0.record(stream)
+        for _ in range(n_u):
+            ug.replay()
+        u1.record(stream)
+        torch.cuda.synchronize()
+        us = u0.elapsed_time(u1) * 1e3 / n_u
+        ubytes = w.batch * w.block_size * Vv * 2
+        unmask = {"vocab": Vv, "us_per_call": round(us, 3), "bytes": ubytes,
+                  "gbs": round(ubytes / (us * 1e-6) / 1e9, 2), "launches_per_call": 2}
+
     # ---- oracle CPU baseline (rank 0, N = 1 only) ----
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
@@ -470,6 +497,7 @@ def run_native(args):
         "e2e": e2e,
         "kv_append": kv_app,
         "backward": bwd,
+        "unmask": unmask,
         "cpu_baseline": cpu,
         "clocks": ck,
     }

@@ -194,6 +194,24 @@ TT_API tt_status_t tt_block_attn_block_causal_backward(tt_plan_t plan, const voi
                                                        float* dq, float* dk_blk, float* dv_blk,
                                                        tt_stream_t stream);
 
+/* Confidence-unmasking step of block sampling (paperfeed.app review of arXiv
+ * 2606.26493, section "Training and sampling": every masked position is predicted in
+ * parallel, each prediction with confidence above gamma = 0.8 is committed, the rest
+ * stay masked for the next step).  For each position (n, s) masked on entry:
+ *   argmax[n, s] = the first index of the largest logit,
+ *   p_max[n, s]  = its softmax probability (fp32);
+ * positions not masked on entry get p_max = 0, argmax = -1 and are not changed.
+ * Then, per sequence, every masked position with p_max > gamma commits
+ * (tokens[n, s] = argmax[n, s], masked[n, s] = 0); when none does and min_one is
+ * non-zero, the masked position with the largest p_max (the first among equals)
+ * commits instead.  n_committed[n] (may be NULL) receives the count.
+ *   logits [B, S, V] bf16 (16-byte aligned); tokens [B, S] int32 and masked [B, S]
+ *   uint8 updated in place; p_max [B, S] fp32 and argmax [B, S] int32 written.
+ * Uses the current device; asynchronous on `stream`; 1 <= S <= 1024. */
+TT_API tt_status_t tt_confidence_unmask(const void* logits, int batch, int block, int vocab, float gamma,
+                                        int min_one, int32_t* tokens, uint8_t* masked, float* p_max,
+                                        int32_t* argmax, int32_t* n_committed, tt_stream_t stream);
+
 /* Committed-block cache update (paperfeed.app review of arXiv 2606.26493, section
  * "The idea: freeze the reader, train the writer": a committed block is ingested by
  * the frozen context tower, "updating its caches").  For every sequence n:

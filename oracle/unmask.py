@@ -29,7 +29,8 @@ def confidence_unmask(logits, tokens, masked, gamma=0.8, min_one=True):
     """logits [B, S, V] (float); tokens [B, S] int; masked [B, S] bool.
 
     Returns (tokens', masked', p [B, S] float64, arg [B, S] int64, n_committed [B]).
-    p and arg are reported for every position; only masked positions can commit.
+    p and arg are reported for the positions masked on entry (p = 0 and arg = -1
+    elsewhere); only those positions can commit.
     """
     x = np.asarray(logits, dtype=np.float64)
     B, S, V = x.shape
@@ -38,6 +39,8 @@ def confidence_unmask(logits, tokens, masked, gamma=0.8, min_one=True):
     p = 1.0 / np.exp(x - m[:, :, None]).sum(axis=2)  # probability of the argmax token
     tok = np.array(tokens, dtype=np.int64, copy=True)
     msk = np.array(masked, dtype=bool, copy=True)
+    p = np.where(msk, p, 0.0)
+    arg = np.where(msk, arg, -1)
     n_commit = np.zeros(B, dtype=np.int64)
     for n in range(B):
         commit = msk[n] & (p[n] > gamma)

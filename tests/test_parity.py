@@ -377,3 +377,35 @@ def test_block_causal_backward_full_sampled():
         assert_parity(dq[:1, sl], rq[:, sl], f"dq block {b}")
         assert_parity(dk[:1, sl], rk[:, sl], f"dk_blk block {b}")
         assert_parity(dv[:1, sl], rv[:, sl], f"dv_blk block {b}")
+
+
+# --- confidence-unmasking step --------------------------------------------------------
+@pytest.mark.parametrize("V", [131072, 1001], ids=["V131072", "V1001-unaligned"])
+@pytest.mark.parametrize("min_one", [True, False])
+def test_confidence_unmask(V, min_one):
+    from oracle import confidence_unmask as oracle_unmask
+    rng = np.random.default_rng(51 + V % 7)
+    B, S = 4, 16
+    x = rng.standard_normal((B, S, V)).astype(np.float32)
+    # a few confident positions (p near 0.95 or 0.5, far from the 0.8 threshold)
+    for (n, s_, boost) in [(0, 3, 30.0), (0, 9, 30.0), (1, 0, 30.0), (2, 5, np.log(V) + 0.2), (3, 15, 30.0)]:
+        x[n, s_, (n * 1000 + s_ * 7) % V] = boost
+    bits = bf16_bits(x)
+    tokens = np.full((B, S), -1, dtype=np.int32)
+    masked = np.ones((B, S), dtype=np.uint8)
+    masked[0, 9] = 0           # already committed: untouched even though confident
+    masked[3, :8] = 0
+    tokens[masked == 0] = 7
+    rt, rm, rp, ra, rn = oracle_unmask(f64(bits), tokens, masked.astype(bool), gamma=0.8, min_one=min_one)
+    # the test inputs keep every decision unambiguous: no masked confidence near 0.8 and, where
+    # the fallback may decide, a unique most confident position
+    assert np.all(np.abs(rp[masked == 1] - 0.8) > 1e-3)
+    dt, dm = torch.from_numpy(tokens).cuda(), torch.from_numpy(masked).cuda()
+    p_max, arg, n_c = ops.confidence_unmask(dev(bits), dt, dm, gamma=0.8, min_one=min_one)
+    torch.cuda.synchronize()
+    assert np.array_equal(arg.cpu().numpy(), ra)
+    gp = p_max.cpu().numpy()
+    assert np.allclose(gp, rp, rtol=1e-4, atol=1e-9)
+    assert np.array_equal(dt.cpu().numpy(), rt)
+    assert np.array_equal(dm.cpu().numpy().astype(bool), rm)
+    assert np.array_equal(n_c.cpu().numpy(), rn)

@@ -16,6 +16,7 @@
 #include "problem.h"
 #include "kv_append.h"
 #include "attn_bwd.h"
+#include "unmask.h"
 #include "errbits.h"
 #include "sched.cuh"
 
@@ -536,6 +537,22 @@ tt_status_t tt_block_attn_block_causal_backward(tt_plan_t plan, const void* q, c
   e = tt::launch_attn_bwd(p, s);
   prof_mark(plan, 2, s, false);
   if (e != cudaSuccess) return cuda_fail(e, "backward kernel launch");
+  return TT_OK;
+}
+
+tt_status_t tt_confidence_unmask(const void* logits, int batch, int block, int vocab, float gamma, int min_one,
+                                 int32_t* tokens, uint8_t* masked, float* p_max, int32_t* argmax, int32_t* n_committed,
+                                 tt_stream_t stream) {
+  if (batch < 0 || block < 1 || block > 1024 || vocab < 1)
+    return fail(TT_ERR_INVALID_ARG, "need batch >= 0, 1 <= block <= 1024, vocab >= 1");
+  if (batch == 0) return TT_OK;
+  if (!logits || !tokens || !masked || !p_max || !argmax) return fail(TT_ERR_INVALID_ARG, "null tensor pointer");
+  if (!aligned16(logits) || (reinterpret_cast<uintptr_t>(tokens) & 3u) || (reinterpret_cast<uintptr_t>(p_max) & 3u) ||
+      (reinterpret_cast<uintptr_t>(argmax) & 3u) || (reinterpret_cast<uintptr_t>(n_committed) & 3u))
+    return fail(TT_ERR_INVALID_ARG, "logits must be 16-byte aligned, the int/float arrays 4-byte aligned");
+  cudaError_t e = tt::launch_confidence_unmask(logits, batch, block, vocab, gamma, min_one ? 1 : 0, tokens, masked,
+                                               p_max, argmax, n_committed, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "confidence unmask launch");
   return TT_OK;
 }
 

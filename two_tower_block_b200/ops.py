@@ -14,7 +14,7 @@ from dataclasses import dataclass
 
 import torch
 
-__all__ = ["TTError", "Plan", "lib", "library_path", "block_attn", "block_attn_block_causal",
+__all__ = ["TTError", "Plan", "lib", "library_path", "block_attn", "block_attn_block_causal", "confidence_unmask",
            "selftest_wait_timeout", "work_split", "KERNEL_AUTO", "KERNEL_TCGEN05", "KERNEL_MMA_SYNC",
            "TT_OK", "TT_ERR_INVALID_ARG", "TT_ERR_UNSUPPORTED", "TT_ERR_CUDA", "TT_ERR_DEVICE_ARG",
            "TT_ERR_TIMEOUT", "EXPORTED_SYMBOLS"]
@@ -32,7 +32,7 @@ EXPORTED_SYMBOLS = [
     "tt_block_attn_block_causal", "tt_block_attn_host", "tt_block_attn_check", "tt_block_attn_profile",
     "tt_block_attn_profile_read", "tt_selftest_wait_timeout", "tt_debug_work_split", "tt_status_string",
     "tt_last_error_detail", "tt_block_attn_noalloc", "tt_selftest_exp2", "tt_kv_append",
-    "tt_block_attn_block_causal_backward",
+    "tt_block_attn_block_causal_backward", "tt_confidence_unmask",
 ]
 
 
@@ -233,6 +233,23 @@ class Plan:
         _check(lib().tt_block_attn_profile_read(self._h, kernel_id, ctypes.byref(n), ctypes.byref(ms)),
                "tt_block_attn_profile_read")
         return n.value, ms.value
+
+
+def confidence_unmask(logits, tokens, masked, gamma=0.8, min_one=True, stream=None):
+    """One unmasking step on CUDA tensors: logits [B,S,V] bf16, tokens [B,S] int32 and
+    masked [B,S] uint8 (updated in place).  Returns (p_max [B,S] fp32, argmax [B,S] int32,
+    n_committed [B] int32)."""
+    B, S, V = logits.shape
+    p_max = torch.empty((B, S), dtype=torch.float32, device=logits.device)
+    arg = torch.empty((B, S), dtype=torch.int32, device=logits.device)
+    n_c = torch.empty((B,), dtype=torch.int32, device=logits.device)
+    lib().tt_confidence_unmask.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float,
+                                           ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                           ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
+    _check(lib().tt_confidence_unmask(_ptr(logits), B, S, V, float(gamma), int(bool(min_one)), _ptr(tokens),
+                                      _ptr(masked), _ptr(p_max), _ptr(arg), _ptr(n_c), _stream(stream)),
+           "tt_confidence_unmask")
+    return p_max, arg, n_c
 
 
 _plans = {}
