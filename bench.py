@@ -158,6 +158,12 @@ def max_over_ranks(pg, value, device=None):
     return float(t.item())
 
 
+def replica_rate(world, units_per_replica, ms_max):
+    """Whole-job rate of `world` replicas that each process `units_per_replica` in a step whose
+    slowest rank took `ms_max` milliseconds: units per second summed over all ranks."""
+    return world * units_per_replica / (ms_max * 1e-3)
+
+
 def workload_cost(wid, inp):
     from two_tower_block_b200.workloads import WORKLOADS, causal_cost, decode_cost
     w = WORKLOADS[wid]
@@ -462,8 +468,8 @@ def run_native(args):
     if rank != 0:
         return 0
     peaks = load_peaks()
-    value = world * cost["bytes"] / (ms_step * 1e-3) / 1e9
-    tflops = world * cost["flops"] / (ms_step * 1e-3) / 1e12
+    value = replica_rate(world, cost["bytes"], ms_step) / 1e9      # ms_step is already the max over ranks
+    tflops = replica_rate(world, cost["flops"], ms_step) / 1e12
     k_ms = ms_k / max(n_k, 1)
     achieved = cost["bytes"] / (k_ms * 1e-3) / 1e9
     bound = "hbm" if w.kind == "decode" else "tensor"
