@@ -72,7 +72,27 @@ def test_null_arguments():
     assert L.tt_block_attn_plan(None, 0, None) == ops.TT_ERR_INVALID_ARG
     assert L.tt_block_attn(None, *([None] * 9)) == ops.TT_ERR_INVALID_ARG
     assert L.tt_block_attn_check(None, None) == ops.TT_ERR_INVALID_ARG
+    assert L.tt_kv_append(None, *([None] * 5), 1, None) == ops.TT_ERR_INVALID_ARG
+    assert L.tt_block_attn_block_causal_backward(None, *([None] * 12)) == ops.TT_ERR_INVALID_ARG
     L.tt_block_attn_plan_destroy(None)  # no-op
+
+
+@pytest.mark.parametrize("B,S,V", [(-1, 16, 10), (1, 0, 10), (1, 1025, 10), (1, 16, 0)])
+def test_confidence_unmask_rejects_bad_shapes_before_the_device(B, S, V):
+    import ctypes
+    L = ops.lib()
+    L.tt_confidence_unmask.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float,
+                                       ctypes.c_int] + [ctypes.c_void_p] * 6
+    assert L.tt_confidence_unmask(None, B, S, V, 0.8, 1, None, None, None, None, None, None) == ops.TT_ERR_INVALID_ARG
+
+
+def test_confidence_unmask_rejects_null_tensors_and_empty_batch_is_a_noop():
+    import ctypes
+    L = ops.lib()
+    L.tt_confidence_unmask.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float,
+                                       ctypes.c_int] + [ctypes.c_void_p] * 6
+    assert L.tt_confidence_unmask(None, 2, 16, 100, 0.8, 1, None, None, None, None, None, None) == ops.TT_ERR_INVALID_ARG
+    assert L.tt_confidence_unmask(None, 0, 16, 100, 0.8, 1, None, None, None, None, None, None) == ops.TT_OK
 
 
 @pytest.mark.parametrize("tiles,C", [
