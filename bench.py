@@ -63,7 +63,8 @@ def load_peaks():
 
 
 def kernel_source_hash(kind: str) -> str:
-    files = {"tcgen05": ["attn_tcgen05.cu"], "mma_sync": ["attn_mma_sync.cu"]}[kind]
+    files = {"tcgen05": ["attn_tcgen05.cu"], "tcgen05_pt": ["attn_tcgen05_pt.cu", "tc_common.cuh"],
+             "tcgen05_2sm": ["attn_tcgen05_2sm.cu", "tc_common.cuh"], "mma_sync": ["attn_mma_sync.cu"]}[kind]
     h = hashlib.sha256()
     for f in files + ["ptx.cuh", "walker.cuh", "problem.h", "sched.cuh"]:
         h.update(open(os.path.join(ROOT, "two_tower_block_b200", "csrc", f), "rb").read())
@@ -287,6 +288,8 @@ def run_native(args):
 
     info = plan.info()
     kname = {1: "tcgen05", 2: "mma_sync"}[info.kernel]
+    if info.kernel == 1 and info.variant in (2, 3):   # the selectable tcgen05 forms have their own sources
+        kname = {2: "tcgen05_pt", 3: "tcgen05_2sm"}[info.variant]
     stream = torch.cuda.current_stream()
     for i in range(max(3, args.warmup)):
         step(i)

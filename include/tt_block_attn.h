@@ -98,6 +98,8 @@ typedef struct {
   int rows_per_unit;       /* S * g, the packed query rows of one (sequence, KV head) */
   size_t workspace_bytes;  /* device scratch owned by the plan                        */
   int sm_count;
+  int variant;             /* tcgen05 kernel form: 0 default, 2 transposed PV, 3 2-SM pairs */
+  int fused_combine;       /* non-zero: the split combine runs in the attention kernel's tail */
 } tt_plan_info;
 
 /* Create a plan: validates the descriptor, picks the kernel and the work split

@@ -391,6 +391,8 @@ tt_status_t tt_block_attn_plan_get_info(tt_plan_t plan, tt_plan_info* info) {
   info->rows_per_unit = plan->R;
   info->workspace_bytes = plan->ws_bytes;
   info->sm_count = plan->sm_count;
+  info->variant = plan->kernel == TT_KERNEL_TCGEN05 ? plan->variant : 0;
+  info->fused_combine = plan->fused_combine ? 1 : 0;
   return TT_OK;
 }
 

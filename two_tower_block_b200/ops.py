@@ -46,7 +46,7 @@ class Desc(ctypes.Structure):
 class PlanInfo(ctypes.Structure):
     _fields_ = [("kernel", ctypes.c_int), ("num_ctas", ctypes.c_int), ("key_tile", ctypes.c_int),
                 ("rows_per_unit", ctypes.c_int), ("workspace_bytes", ctypes.c_size_t),
-                ("sm_count", ctypes.c_int)]
+                ("sm_count", ctypes.c_int), ("variant", ctypes.c_int), ("fused_combine", ctypes.c_int)]
 
 
 _lib = None
