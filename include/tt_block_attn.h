@@ -25,10 +25,15 @@
  * c_{<b} and on itself): block b of a length-N sequence attends to context
  * positions [0, S*b) and to its own block positions [S*b, S*b+S).
  *
+ * Besides the two attention entry points, the library carries the steps next to
+ * them in a denoising loop: the block-causal backward (gradients for training),
+ * the committed-block cache update and the confidence-unmasking step.
+ *
  * Conventions shared by every entry point
  *   - Tensors are dense, row-major, device memory owned by the caller.
- *     q, k_*, v_* are bf16; out and lse are fp32; ctx_lens is int32.
- *     Every tensor pointer must be 16-byte aligned.
+ *     q, k_*, v_* (and the backward's dout) are bf16; out, lse and gradients
+ *     are fp32; ctx_lens is int32.  Every tensor pointer must be 16-byte
+ *     aligned (the unmasking step's int / float arrays: 4-byte).
  *   - Calls are asynchronous and ordered on `stream`; none synchronises the
  *     host except tt_block_attn_check and tt_block_attn_profile_read.
  *   - A plan may be used by one stream at a time (it owns scratch memory).
@@ -62,7 +67,7 @@ typedef enum {
   TT_ERR_INVALID_ARG = 1,   /* null / misaligned pointer, bad descriptor or size     */
   TT_ERR_UNSUPPORTED = 2,   /* valid but not implemented (e.g. head_dim 96)          */
   TT_ERR_CUDA = 3,          /* a CUDA runtime call or a kernel launch failed         */
-  TT_ERR_DEVICE_ARG = 4,    /* seen on the device: ctx_lens[n] < 0 or > capacity     */
+  TT_ERR_DEVICE_ARG = 4,    /* seen on the device: a ctx_lens value out of range     */
   TT_ERR_TIMEOUT = 5        /* seen on the device: a pipeline wait ran out its limit */
 } tt_status_t;
 
