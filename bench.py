@@ -49,6 +49,7 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-paged", action="store_true", help="skip the paged-cache decode measurement")
     ap.add_argument("--num-ctas", type=int, default=0, help="work ranges (0: the plan's choice)")
     return ap.parse_args()
 
@@ -370,6 +371,63 @@ def run_native(args):
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": round(ms_e2e, 4),
                "steps": n_e2e}
 
+    # ---- the same decode over a paged cache: 64-row pages in a shuffled pool ----
+    paged = None
+    if w.kind == "decode" and not args.no_paged:
+        from two_tower_block_b200.workloads import make_paged
+        P = 64
+        pc = make_paged(inp, P, seed=w.seed, spare_pages=0, fill_bits=0)
+        ptab = torch.from_numpy(pc.page_table).to(dev)
+        pbase = [to_dev(pc.k_pages), to_dev(pc.v_pages)]
+        pcopies = [pbase] + [[t.clone() for t in pbase] for _ in range(n_copies - 1)]
+        pplan = ops.Plan(w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_size, ctx_capacity=0,
+                         kernel=kernel, num_ctas=args.num_ctas, device=local)
+
+        def pstep(i):
+            c, pk = copies[i % n_copies], pcopies[i % n_copies]
+            pplan.block_attn_paged(c[0], pk[0], pk[1], ptab, c[3], c[4], lens, out=out, lse=lse)
+        for i in range(max(3, args.warmup)):
+            pstep(i)
+        pplan.check()
+        pgraphs = None
+        if not args.no_graph:
+            pgraphs = []
+            for i in range(n_copies):
+                gph = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(gph):
+                    pstep(i)
+                pgraphs.append(gph)
+            for gph in pgraphs:
+                gph.replay()
+        torch.cuda.synchronize()
+        p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        p0.record(stream)
+        for i in range(args.steps):
+            if pgraphs:
+                pgraphs[i % n_copies].replay()
+            else:
+                pstep(i)
+        p1.record(stream)
+        torch.cuda.synchronize()
+        pplan.profile(True)
+        for i in range(args.steps):
+            pstep(i)
+        torch.cuda.synchronize()
+        n_pk, ms_pk = pplan.profile_read(0)
+        n_pc, _ = pplan.profile_read(1) if info.num_ctas > 1 else (0, 0.0)
+        pplan.profile(False)
+        pplan.check()
+        ms_pstep = max_over_ranks(pg, p0.elapsed_time(p1) / args.steps, dev)
+        pk_ms = ms_pk / max(n_pk, 1)
+        tbytes = int(sum(-(-int(L) // P) for L in inp.ctx_lens)) * 4 * w.num_kv_heads   # table entries read
+        pbytes = cost["bytes"] + tbytes
+        paged = {"page_size": P, "pool_pages": int(pc.k_pages.shape[0]), "ms_per_step": round(ms_pstep, 5),
+                 "value": round(replica_rate(world, pbytes, ms_pstep) / 1e9, 3), "unit": "GB/s",
+                 "kernel_ms": round(pk_ms, 5), "kernel_gbs": round(pbytes / (pk_ms * 1e-3) / 1e9, 2),
+                 "kernel_time_vs_contiguous": round(pk_ms / (ms_k / max(n_k, 1)), 4),
+                 "launches_per_step": (n_pk + n_pc) // max(args.steps, 1)}
+        del pcopies, pbase
+
     # ---- block-causal backward at this workload's shape (training workloads) ----
     bwd = None
     if w.kind == "causal":
@@ -505,6 +563,7 @@ def run_native(args):
         "num_ctas": info.num_ctas,
         "e2e": e2e,
         "kv_append": kv_app,
+        "paged": paged,
         "backward": bwd,
         "unmask": unmask,
         "cpu_baseline": cpu,

@@ -135,6 +135,35 @@ TT_API tt_status_t tt_block_attn(tt_plan_t plan, const void* q, const void* k_ct
                           const void* k_blk, const void* v_blk, const int32_t* ctx_lens,
                           float* out, float* lse, tt_stream_t stream);
 
+/* Decode over a PAGED context cache: the serving form, where the context tower's
+ * layer-i cache of every sequence lives in fixed-size pages drawn from one shared pool
+ * (blocks are committed one after another and contexts differ widely in length, so a
+ * contiguous Lcap slab per sequence would waste memory).  Same attention as
+ * tt_block_attn; only the addressing of the context keys and values differs.
+ *   k_pages    [num_pages, Hkv, page_size, D] bf16  key pool (device)
+ *   v_pages    [num_pages, Hkv, page_size, D] bf16  value pool (device)
+ *   page_table [B, pages_per_seq]             int32 pool page of each sequence's
+ *              logical page: position l of sequence n is row l % page_size of page
+ *              page_table[n][l / page_size] (device, read-only)
+ *   q, k_blk, v_blk, ctx_lens, out, lse       as tt_block_attn, with
+ *              0 <= ctx_lens[n] <= pages_per_seq * page_size
+ * page_size is a power of two in [16, 65536]; the plan's ctx_capacity is not used.
+ * Only the entries page_table[n][0 .. ceil(L_n / page_size)) are read; every one of
+ * them must lie in [0, num_pages): a page outside the pool reads as zeros and is
+ * flagged TT_ERR_DEVICE_ARG (as are out-of-range ctx_lens, which are clamped).
+ * pages_per_seq == 0 means no context (k_pages / v_pages / page_table may be NULL).
+ * Runs the default tcgen05 kernel (whatever TT_TCGEN05_VARIANT selects for
+ * tt_block_attn) or the mma.sync kernel, as the plan chose; the caller owns all
+ * buffers, nothing is allocated.  TT_ERR_INVALID_ARG for a bad page_size, negative
+ * counts, a NULL pointer that is needed or a misaligned one (16 bytes for the bf16
+ * and fp32 tensors, 4 for the int32 arrays); TT_ERR_UNSUPPORTED when a pool or a
+ * logical capacity holds 2^31 rows or more. */
+TT_API tt_status_t tt_block_attn_paged(tt_plan_t plan, const void* q, const void* k_pages,
+                                const void* v_pages, const int32_t* page_table, int32_t num_pages,
+                                int32_t page_size, int32_t pages_per_seq, const void* k_blk,
+                                const void* v_blk, const int32_t* ctx_lens, float* out, float* lse,
+                                tt_stream_t stream);
+
 /* Block-causal training / prefill form over whole sequences of length N = seq_len.
  *   q      [B, N, Hq, D]  bf16      out [B, N, Hq, D] fp32
  *   k_ctx  [B, Hkv, N, D] bf16 (context tower over the clean sequence), v_ctx likewise

@@ -188,8 +188,20 @@ tt_status_t launch_all(tt_plan_t plan, const tt::Problem& p, cudaStream_t s) {
           !encode_bf16(&maps.v_blk, p.v_blk, 3, dims, str, box))
         return fail(TT_ERR_CUDA, "tensor map (block kv) encode failed");
     }
-    // k_ctx / v_ctx viewed as [B*Hkv*stride rows][D]; box = key_tile rows x 64 dims
-    if ((uint64_t)p.B * p.Hkv * p.ctx_stride > 0) {
+    // paged: k_ctx / v_ctx are pools viewed as [num_pages*Hkv*page_size rows][D]; box =
+    // min(page_size, key_tile) rows x 64 dims (one page's slice of a tile)
+    if (p.page_table && (uint64_t)p.num_pages * p.Hkv * p.ctx_stride > 0) {
+      uint64_t dims[2] = {D, ((uint64_t)p.num_pages * p.Hkv) << p.page_shift};
+      uint64_t str[1] = {D * 2};
+      uint32_t box[2] = {64, std::min(1u << p.page_shift, kt)};
+      if (!encode_bf16(&maps.k_ctx, p.k_ctx, 2, dims, str, box) ||
+          !encode_bf16(&maps.v_ctx, p.v_ctx, 2, dims, str, box))
+        return fail(TT_ERR_CUDA, "tensor map (paged context kv) encode failed");
+    } else if (p.page_table) {
+      maps.k_ctx = maps.k_blk;  // never read: no context tiles exist
+      maps.v_ctx = maps.v_blk;
+    } else if ((uint64_t)p.B * p.Hkv * p.ctx_stride > 0) {
+      // k_ctx / v_ctx viewed as [B*Hkv*stride rows][D]; box = key_tile rows x 64 dims
       uint64_t dims[2] = {D, (uint64_t)p.B * p.Hkv * p.ctx_stride};
       uint64_t str[1] = {D * 2};
       uint32_t box[2] = {64, kt};
@@ -414,6 +426,49 @@ tt_status_t tt_block_attn(tt_plan_t plan, const void* q, const void* k_ctx, cons
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.k_ctx = static_cast<const __nv_bfloat16*>(k_ctx);
   p.v_ctx = static_cast<const __nv_bfloat16*>(v_ctx);
+  p.k_blk = static_cast<const __nv_bfloat16*>(k_blk);
+  p.v_blk = static_cast<const __nv_bfloat16*>(v_blk);
+  p.ctx_lens = ctx_lens;
+  p.out = out;
+  p.lse = lse;
+  return launch_all(plan, p, reinterpret_cast<cudaStream_t>(stream));
+}
+
+tt_status_t tt_block_attn_paged(tt_plan_t plan, const void* q, const void* k_pages, const void* v_pages,
+                                const int32_t* page_table, int32_t num_pages, int32_t page_size,
+                                int32_t pages_per_seq, const void* k_blk, const void* v_blk, const int32_t* ctx_lens,
+                                float* out, float* lse, tt_stream_t stream) {
+  if (!plan) return fail(TT_ERR_INVALID_ARG, "null plan");
+  const tt_block_attn_desc& d = plan->desc;
+  if (page_size < 16 || page_size > (1 << 16) || (page_size & (page_size - 1)))
+    return fail(TT_ERR_INVALID_ARG, "page_size must be a power of two in [16, 65536]");
+  if (num_pages < 0 || pages_per_seq < 0) return fail(TT_ERR_INVALID_ARG, "negative num_pages or pages_per_seq");
+  if ((long long)pages_per_seq * page_size > (1ll << 31) - 1 ||
+      (long long)num_pages * d.num_kv_heads * page_size > (1ll << 31) - 1)
+    return fail(TT_ERR_UNSUPPORTED, "page pool or page table too large (rows beyond 2^31)");
+  if (d.batch == 0) return TT_OK;
+  if (!q || !k_blk || !v_blk || !ctx_lens || !out) return fail(TT_ERR_INVALID_ARG, "null tensor pointer");
+  if (pages_per_seq > 0 && (!page_table || !k_pages || !v_pages || num_pages < 1))
+    return fail(TT_ERR_INVALID_ARG, "pages_per_seq > 0 needs a page table and non-empty pools");
+  if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned16(k_blk) || !aligned16(v_blk) ||
+      !aligned16(out) || !aligned16(lse) || (reinterpret_cast<uintptr_t>(ctx_lens) & 3u) ||
+      (reinterpret_cast<uintptr_t>(page_table) & 3u))
+    return fail(TT_ERR_INVALID_ARG, "tensor pointer not 16-byte aligned");
+  DeviceGuard guard(plan->device);
+  tt::Problem p = base_problem(plan);
+  p.mode = tt::kDecode;
+  p.NB = 1;
+  p.variant = 0;  // the paged loads live in the default tcgen05 kernel (and the mma.sync one)
+  p.ctx_stride = pages_per_seq * page_size;
+  int shift = 0;
+  while ((1 << shift) < page_size) ++shift;
+  p.page_shift = shift;
+  p.pages_per_seq = pages_per_seq;
+  p.num_pages = num_pages;
+  p.page_table = pages_per_seq > 0 ? page_table : nullptr;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.k_ctx = static_cast<const __nv_bfloat16*>(k_pages);
+  p.v_ctx = static_cast<const __nv_bfloat16*>(v_pages);
   p.k_blk = static_cast<const __nv_bfloat16*>(k_blk);
   p.v_blk = static_cast<const __nv_bfloat16*>(v_blk);
   p.ctx_lens = ctx_lens;

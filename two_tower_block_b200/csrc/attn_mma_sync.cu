@@ -70,7 +70,7 @@ __global__ void __launch_bounds__(kThreads) attn_mma_sync_kernel(const Problem p
       const TileKeys tk = tile_keys(p, x, i);
       for (int e = tid; e < kKeys * CH; e += kThreads) {
         const int r = e / CH, ch = e - (e / CH) * CH;
-        const bool valid = r < tk.count;
+        bool valid = r < tk.count;
         const __nv_bfloat16* ks = p.k_blk;
         const __nv_bfloat16* vs = p.v_blk;
         if (valid) {
@@ -78,10 +78,17 @@ __global__ void __launch_bounds__(kThreads) attn_mma_sync_kernel(const Problem p
             const size_t off = ((size_t)(x.ns * p.S + tk.first + r) * p.Hkv + x.h) * D + ch * 8;
             ks = p.k_blk + off;
             vs = p.v_blk + off;
-          } else {
+          } else if (!p.page_table) {
             const size_t off = ((size_t)(x.n * p.Hkv + x.h) * p.ctx_stride + tk.first + r) * D + ch * 8;
             ks = p.k_ctx + off;
             vs = p.v_ctx + off;
+          } else {
+            const int row = paged_row(p, x.n, x.h, tk.first + r);  // -1: page outside the pool
+            valid = row >= 0;  // a bad page reads as zeros
+            if (valid) {
+              ks = p.k_ctx + (size_t)row * D + ch * 8;
+              vs = p.v_ctx + (size_t)row * D + ch * 8;
+            }
           }
         }
         cp_async_16(smem_u32(sK + (buf * kKeys + r) * LDS + ch * 8), ks, valid);

@@ -238,9 +238,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       ++q_it;
       const int ctx_row0 = (x.n * p.Hkv + x.h) * p.ctx_stride;
+      // paged cache: a context tile is loaded in slices of psub rows, one per page (pages of
+      // at least NK keys hold whole tiles); slices past the tile's last key are not loaded
+      const int psub = p.page_table ? min(1 << p.page_shift, NK) : NK;
       for (int i = sg.lo; i < sg.hi && ok; ++i) {
         const TileKeys tk = tile_keys(p, x, i);
-        const int box_rows = tk.is_blk ? min(p.S, NK) : NK;
+        const int box_rows = tk.is_blk ? min(p.S, NK) : (p.page_table ? ceil_div(tk.count, psub) * psub : NK);
         const uint32_t bytes = (uint32_t)(box_rows * kRowBytes * C::kHalves);
         for (int kv = 0; kv < 2 && ok; ++kv, ++it) {
           const int s = it % C::kStages;
@@ -255,8 +258,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive_expect_tx(bar, bytes);
             for (int hf = 0; hf < C::kHalves; ++hf) {
               const uint32_t dst = slot + hf * (NK * kRowBytes);
-              if (tk.is_blk) tma_load_3d(dst, m, bar, hf * 64, x.h, x.ns * p.S + tk.first);
-              else tma_load_2d(dst, m, bar, hf * 64, ctx_row0 + tk.first);
+              if (tk.is_blk) {
+                tma_load_3d(dst, m, bar, hf * 64, x.h, x.ns * p.S + tk.first);
+              } else if (!p.page_table) {
+                tma_load_2d(dst, m, bar, hf * 64, ctx_row0 + tk.first);
+              } else {
+                // a page outside the pool reads as zeros (row coordinate past the pool's end)
+                for (int r = 0; r < box_rows; r += psub) {
+                  const int row = paged_row(p, x.n, x.h, tk.first + r);
+                  tma_load_2d(dst + r * kRowBytes, m, bar, hf * 64, row < 0 ? (p.num_pages * p.Hkv) << p.page_shift : row);
+                }
+              }
             }
           }
           if (fix) {

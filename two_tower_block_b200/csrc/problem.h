@@ -51,6 +51,14 @@ struct Problem {
   // (a counter that only grows) and combine the cut units themselves; null: the
   // separate combine kernel runs instead
   unsigned long long* grid_bar;
+  // paged context cache (decode only; null page_table: contiguous k_ctx / v_ctx).
+  // k_ctx / v_ctx then point at pools [num_pages][Hkv][page_size][D]; context position
+  // pos of sequence n sits in page page_table[n * pages_per_seq + (pos >> page_shift)]
+  // at row pos & (page_size - 1).  ctx_stride = pages_per_seq * page_size.
+  const int* page_table;
+  int page_shift;       // log2(page_size); page_size is a power of two >= 16
+  int pages_per_seq;
+  int num_pages;
 };
 
 // Host launchers (each returns the cudaError_t of its launch).

@@ -175,4 +175,16 @@ __device__ __forceinline__ TileKeys tile_keys(const Problem& p, const Unit& x, i
   return k;
 }
 
+// Pool row (of the [num_pages * Hkv * page_size] rows of k_ctx / v_ctx) holding context
+// position pos of (n, h) in a paged cache; -1, reported as a device argument error, when
+// the page table names a page outside [0, num_pages).
+__device__ __forceinline__ int paged_row(const Problem& p, int n, int h, int pos) {
+  const int page = __ldg(p.page_table + (size_t)n * p.pages_per_seq + (pos >> p.page_shift));
+  if (page < 0 || page >= p.num_pages) {
+    raise_error(p.err_word, kErrDeviceArg);
+    return -1;
+  }
+  return ((page * p.Hkv + h) << p.page_shift) + (pos & ((1 << p.page_shift) - 1));
+}
+
 }  // namespace tt

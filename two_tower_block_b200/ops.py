@@ -32,7 +32,7 @@ EXPORTED_SYMBOLS = [
     "tt_block_attn_block_causal", "tt_block_attn_host", "tt_block_attn_check", "tt_block_attn_profile",
     "tt_block_attn_profile_read", "tt_selftest_wait_timeout", "tt_debug_work_split", "tt_status_string",
     "tt_last_error_detail", "tt_block_attn_noalloc", "tt_selftest_exp2", "tt_kv_append",
-    "tt_block_attn_block_causal_backward", "tt_confidence_unmask",
+    "tt_block_attn_block_causal_backward", "tt_confidence_unmask", "tt_block_attn_paged",
 ]
 
 
@@ -67,6 +67,7 @@ def lib() -> ctypes.CDLL:
     L.tt_block_attn_plan_get_info.argtypes = [vp, ctypes.POINTER(PlanInfo)]
     L.tt_block_attn.argtypes = [vp] * 10
     L.tt_block_attn_block_causal.argtypes = [vp] * 9
+    L.tt_block_attn_paged.argtypes = [vp, vp, vp, vp, vp, i, i, i, vp, vp, vp, vp, vp, vp]
     L.tt_block_attn_host.argtypes = [vp] * 10
     L.tt_block_attn_check.argtypes = [vp, vp]
     L.tt_block_attn_profile.argtypes = [vp, i]
@@ -170,6 +171,23 @@ class Plan:
             lse = torch.empty((s.batch, s.q_heads, s.block), dtype=torch.float32, device=q.device)
         _check(lib().tt_block_attn(self._h, _ptr(q), _ptr(k_ctx), _ptr(v_ctx), _ptr(k_blk), _ptr(v_blk),
                                    _ptr(ctx_lens), _ptr(out), _ptr(lse), _stream(stream)), "tt_block_attn")
+        return (out, lse) if want_lse or lse is not None else out
+
+    def block_attn_paged(self, q, k_pages, v_pages, page_table, k_blk, v_blk, ctx_lens, out=None, lse=None,
+                         stream=None, want_lse=False):
+        """Decode over a paged context cache: k_pages / v_pages [num_pages, Hkv, P, D] bf16
+        pools, page_table [B, pages_per_seq] int32 (device); P = k_pages.shape[2]."""
+        s = self.shape
+        if out is None:
+            out = torch.empty((s.batch, s.block, s.q_heads, s.head_dim), dtype=torch.float32, device=q.device)
+        if lse is None and want_lse:
+            lse = torch.empty((s.batch, s.q_heads, s.block), dtype=torch.float32, device=q.device)
+        num_pages, _, page_size, _ = k_pages.shape
+        pages_per_seq = page_table.shape[1] if page_table is not None and page_table.dim() == 2 else 0
+        _check(lib().tt_block_attn_paged(self._h, _ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(page_table),
+                                         int(num_pages), int(page_size), int(pages_per_seq), _ptr(k_blk),
+                                         _ptr(v_blk), _ptr(ctx_lens), _ptr(out), _ptr(lse), _stream(stream)),
+               "tt_block_attn_paged")
         return (out, lse) if want_lse or lse is not None else out
 
     def block_attn_host(self, q, k_ctx, v_ctx, k_blk, v_blk, ctx_lens, out, lse=None, stream=None):

@@ -201,3 +201,41 @@ def causal_cost(B, N, S, Hq, Hkv, D, out_bytes=4):
     qb = B * N * Hq * D * 2
     ob = B * N * Hq * D * out_bytes
     return {"bytes": kv + qb + ob, "kv_bytes": kv, "flops": flops}
+
+
+@dataclass
+class PagedCache:
+    """A decode cache laid out as a shared page pool (bf16 bit patterns)."""
+    k_pages: np.ndarray      # [num_pages, Hkv, P, D] uint16
+    v_pages: np.ndarray
+    page_table: np.ndarray   # [B, pages_per_seq] int32; entries past ceil(L_n / P) are -1
+    page_size: int
+
+
+def make_paged(inp: DecodeInputs, page_size: int, seed: int, spare_pages: int = 3,
+               fill_bits: int = 0x7FC0) -> PagedCache:
+    """Scatter the first L_n rows of every sequence of ``inp`` into pages of ``page_size``
+    rows drawn in a shuffled order from one pool.  Rows past L_n inside a sequence's last
+    page and ``spare_pages`` pages that no sequence owns hold ``fill_bits`` (bf16 NaN by
+    default), so any read of them shows; unused table entries are -1."""
+    rng = np.random.default_rng(seed)
+    B, Hkv, Lcap, D = inp.k_ctx.shape
+    P = page_size
+    per = -(-Lcap // P) if Lcap else 0
+    need = [-(-int(L) // P) for L in inp.ctx_lens]
+    num_pages = sum(need) + spare_pages
+    order = rng.permutation(num_pages)
+    k_pages = np.full((num_pages, Hkv, P, D), fill_bits, dtype=np.uint16)
+    v_pages = np.full_like(k_pages, fill_bits)
+    table = np.full((B, per), -1, dtype=np.int32)
+    nxt = 0
+    for n in range(B):
+        L = int(inp.ctx_lens[n])
+        for i in range(need[n]):
+            pg = int(order[nxt])
+            nxt += 1
+            table[n, i] = pg
+            rows = min(P, L - i * P)
+            k_pages[pg, :, :rows] = inp.k_ctx[n, :, i * P:i * P + rows]
+            v_pages[pg, :, :rows] = inp.v_ctx[n, :, i * P:i * P + rows]
+    return PagedCache(k_pages, v_pages, table, P)
