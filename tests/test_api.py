@@ -74,6 +74,8 @@ def test_null_arguments():
     assert L.tt_block_attn_check(None, None) == ops.TT_ERR_INVALID_ARG
     assert L.tt_kv_append(None, *([None] * 5), 1, None) == ops.TT_ERR_INVALID_ARG
     assert L.tt_block_attn_block_causal_backward(None, *([None] * 12)) == ops.TT_ERR_INVALID_ARG
+    assert L.tt_block_attn_paged(None, None, None, None, None, 0, 64, 0, None, None, None, None, None,
+                                 None) == ops.TT_ERR_INVALID_ARG
     L.tt_block_attn_plan_destroy(None)  # no-op
 
 
@@ -131,3 +133,15 @@ def test_no_device_plan_creation_reports_cuda_error():
     st = ops.lib().tt_block_attn_plan(ctypes.byref(desc), 0, ctypes.byref(h))
     assert st in (ops.TT_ERR_CUDA, ops.TT_ERR_INVALID_ARG)
     assert not h.value
+
+
+@pytest.mark.parametrize("page_size,num_pages,pages_per_seq", [
+    (0, 1, 1), (8, 1, 1), (48, 1, 1), (1 << 17, 1, 1), (-64, 1, 1), (64, -1, 1), (64, 1, -1)])
+def test_paged_rejects_bad_page_geometry_before_the_device(page_size, num_pages, pages_per_seq):
+    """Page size must be a power of two in [16, 65536] and the counts non-negative; the
+    check precedes every use of the plan or the device."""
+    L = ops.lib()
+    st = L.tt_block_attn_paged(None, None, None, None, None, num_pages, page_size, pages_per_seq, None, None, None,
+                               None, None, None)
+    assert st == ops.TT_ERR_INVALID_ARG
+    assert b"page" in L.tt_last_error_detail()

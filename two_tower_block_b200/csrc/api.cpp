@@ -438,11 +438,11 @@ tt_status_t tt_block_attn_paged(tt_plan_t plan, const void* q, const void* k_pag
                                 const int32_t* page_table, int32_t num_pages, int32_t page_size,
                                 int32_t pages_per_seq, const void* k_blk, const void* v_blk, const int32_t* ctx_lens,
                                 float* out, float* lse, tt_stream_t stream) {
-  if (!plan) return fail(TT_ERR_INVALID_ARG, "null plan");
-  const tt_block_attn_desc& d = plan->desc;
   if (page_size < 16 || page_size > (1 << 16) || (page_size & (page_size - 1)))
     return fail(TT_ERR_INVALID_ARG, "page_size must be a power of two in [16, 65536]");
   if (num_pages < 0 || pages_per_seq < 0) return fail(TT_ERR_INVALID_ARG, "negative num_pages or pages_per_seq");
+  if (!plan) return fail(TT_ERR_INVALID_ARG, "null plan");
+  const tt_block_attn_desc& d = plan->desc;
   if ((long long)pages_per_seq * page_size > (1ll << 31) - 1 ||
       (long long)num_pages * d.num_kv_heads * page_size > (1ll << 31) - 1)
     return fail(TT_ERR_UNSUPPORTED, "page pool or page table too large (rows beyond 2^31)");
