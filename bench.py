@@ -50,6 +50,7 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-paged", action="store_true", help="skip the paged-cache decode measurement")
+    ap.add_argument("--page-size", type=int, default=64, help="rows per page of the paged-cache measurement")
     ap.add_argument("--num-ctas", type=int, default=0, help="work ranges (0: the plan's choice)")
     return ap.parse_args()
 
@@ -371,11 +372,11 @@ def run_native(args):
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": round(ms_e2e, 4),
                "steps": n_e2e}
 
-    # ---- the same decode over a paged cache: 64-row pages in a shuffled pool ----
+    # ---- the same decode over a paged cache: pages of --page-size rows in a shuffled pool ----
     paged = None
     if w.kind == "decode" and not args.no_paged:
         from two_tower_block_b200.workloads import make_paged
-        P = 64
+        P = args.page_size
         pc = make_paged(inp, P, seed=w.seed, spare_pages=0, fill_bits=0)
         ptab = torch.from_numpy(pc.page_table).to(dev)
         pbase = [to_dev(pc.k_pages), to_dev(pc.v_pages)]
