@@ -46,3 +46,29 @@ def test_paged_attention_equals_contiguous():
     o1, l1 = block_attn(q, k_ctx, v_ctx, k_blk, v_blk, lens)
     o2, l2 = block_attn_paged(q, kp, vp, table, k_blk, v_blk, lens, L)
     assert np.allclose(o1, o2, atol=1e-14) and np.allclose(l1, l2, atol=1e-14)
+
+
+def test_make_paged_places_rows_and_fills_the_rest():
+    """The pool builder the GPU tests use: row l of sequence n sits at row l % P of page
+    table[n][l // P]; unused entries are -1; spare pages and rows past L_n hold the fill."""
+    from two_tower_block_b200.workloads import make_decode, make_paged
+    inp = make_decode(3, 4, 4, 2, 64, 100, seed=9, ctx_lens=[100, 0, 33])
+    P = 16
+    pc = make_paged(inp, P, seed=4, spare_pages=2, fill_bits=0x7FC0)
+    need = [-(-int(L) // P) for L in inp.ctx_lens]
+    assert pc.k_pages.shape == (sum(need) + 2, 2, P, 64) and pc.page_table.shape == (3, 7)
+    owned = set()
+    for n, L in enumerate(inp.ctx_lens):
+        assert (pc.page_table[n, need[n]:] == -1).all()
+        for l in range(int(L)):
+            pg = pc.page_table[n, l // P]
+            assert np.array_equal(pc.k_pages[pg, :, l % P], inp.k_ctx[n, :, l])
+            assert np.array_equal(pc.v_pages[pg, :, l % P], inp.v_ctx[n, :, l])
+        for i in range(need[n]):
+            owned.add(int(pc.page_table[n, i]))
+        last = pc.page_table[n, need[n] - 1] if need[n] else None
+        if last is not None:
+            assert (pc.k_pages[last, :, int(L) - (need[n] - 1) * P:] == 0x7FC0).all()
+    assert len(owned) == sum(need)                      # no page is shared
+    spare = sorted(set(range(pc.k_pages.shape[0])) - owned)
+    assert len(spare) == 2 and (pc.k_pages[spare] == 0x7FC0).all() and (pc.v_pages[spare] == 0x7FC0).all()
