@@ -145,3 +145,70 @@ def test_paged_rejects_bad_page_geometry_before_the_device(page_size, num_pages,
                                None, None, None)
     assert st == ops.TT_ERR_INVALID_ARG
     assert b"page" in L.tt_last_error_detail()
+
+
+def _shape_only_plan(**kw):
+    """A Plan object with a shape but no library handle: the binding's argument checks
+    run before any library call, so they can be exercised without a GPU."""
+    p = object.__new__(ops.Plan)
+    d = dict(batch=2, q_heads=8, kv_heads=2, head_dim=64, block=4, ctx_capacity=32, seq_len=0)
+    d.update(kw)
+    p.shape = ops.Shape(**d)
+    p.device = 0
+    p._h = None
+    return p
+
+
+def test_binding_rejects_wrong_dtype_and_size_before_the_library():
+    import torch
+    plan = _shape_only_plan()
+    B, S, Hq, Hkv, D, L = 2, 4, 8, 2, 64, 32
+    q = torch.zeros(B, S, Hq, D, dtype=torch.bfloat16)
+    kc = torch.zeros(B, Hkv, L, D, dtype=torch.bfloat16)
+    kb = torch.zeros(B, S, Hkv, D, dtype=torch.bfloat16)
+    lens = torch.zeros(B, dtype=torch.int32)
+    out = torch.zeros(B, S, Hq, D)
+    with pytest.raises(TypeError, match="q: dtype"):              # fp16 is not bf16
+        plan.block_attn(q.half(), kc, kc, kb, kb, lens, out=out)
+    with pytest.raises(ValueError, match="k_blk: .* elements"):   # one KV head short
+        plan.block_attn(q, kc, kc, kb[:, :, :1], kb, lens, out=out)
+    with pytest.raises(ValueError, match="k_ctx: .* elements"):   # capacity 16, plan has 32
+        plan.block_attn(q, kc[:, :, :16], kc, kb, kb, lens, out=out)
+    with pytest.raises(TypeError, match="ctx_lens"):              # int64 lengths
+        plan.block_attn(q, kc, kc, kb, kb, lens.long(), out=out)
+    with pytest.raises(TypeError, match="out"):                   # bf16 output
+        plan.block_attn(q, kc, kc, kb, kb, lens, out=out.bfloat16())
+    with pytest.raises(ValueError, match="cuda:0"):               # right sizes, host memory
+        plan.block_attn(q, kc, kc, kb, kb, lens, out=out)
+
+
+def test_binding_checks_paged_pool_and_table_shapes():
+    import torch
+    plan = _shape_only_plan(ctx_capacity=0)
+    B, S, Hq, Hkv, D = 2, 4, 8, 2, 64
+    q = torch.zeros(B, S, Hq, D, dtype=torch.bfloat16)
+    kb = torch.zeros(B, S, Hkv, D, dtype=torch.bfloat16)
+    lens = torch.zeros(B, dtype=torch.int32)
+    out = torch.zeros(B, S, Hq, D)
+    pool = torch.zeros(5, Hkv, 16, D, dtype=torch.bfloat16)
+    table = torch.zeros(B, 3, dtype=torch.int32)
+    with pytest.raises(ValueError, match="k_pages: shape"):       # KV heads and head_dim swapped
+        plan.block_attn_paged(q, pool.view(5, D, 16, Hkv), pool, table, kb, kb, lens, out=out)
+    with pytest.raises(ValueError, match="v_pages: .* elements"):
+        plan.block_attn_paged(q, pool, pool[:4], table, kb, kb, lens, out=out)
+    with pytest.raises(ValueError, match="page_table: shape"):    # one row per sequence
+        plan.block_attn_paged(q, pool, pool, table[:1], kb, kb, lens, out=out)
+    with pytest.raises(TypeError, match="page_table"):
+        plan.block_attn_paged(q, pool, pool, table.long(), kb, kb, lens, out=out)
+
+
+def test_binding_accepts_bf16_bit_patterns_as_two_byte_integers():
+    import torch
+    ops._arg(torch.zeros(6, dtype=torch.int16), "x", 6, "bf16", None)
+    ops._arg(torch.zeros(6, dtype=torch.bfloat16), "x", 6, "bf16", None)
+    with pytest.raises(TypeError):
+        ops._arg(torch.zeros(6, dtype=torch.float16), "x", 6, "bf16", None)
+    ops._arg(torch.zeros(1, dtype=torch.int32), "status", 1, "w32", None)
+    with pytest.raises(TypeError):
+        ops._arg(torch.zeros(1, dtype=torch.float32), "status", 1, "w32", None)
+    ops._arg(torch.zeros(3), "out", 3, "f32", "host")

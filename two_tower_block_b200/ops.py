@@ -111,6 +111,38 @@ def _ptr(t):
     return ctypes.c_void_p(int(t))
 
 
+def _arg(t, name, numel, kind, device):
+    """Check one tensor argument before its address reaches the library, whose kernels
+    trust every size: ``kind`` "bf16" (any 2-byte type: bf16 values or their bit
+    patterns), "f32", "i32", "w32" (any 4-byte integer) or "u8" (any 1-byte type); ``numel`` the element count the
+    layout needs; ``device`` a CUDA ordinal, "host", or None (not checked).  None and raw integer addresses
+    are passed through (the library rejects a null pointer it needs)."""
+    if not isinstance(t, torch.Tensor):
+        return
+    ok = {"bf16": t.element_size() == 2 and not t.is_floating_point() or t.dtype == torch.bfloat16,
+          "f32": t.dtype == torch.float32, "i32": t.dtype == torch.int32,
+          "w32": t.element_size() == 4 and not t.is_floating_point(),
+          "u8": t.element_size() == 1}[kind]
+    if not ok:
+        raise TypeError(f"{name}: dtype {t.dtype} where {kind} is expected")
+    if t.numel() != numel:
+        raise ValueError(f"{name}: {t.numel()} elements where the plan's shape needs {numel}")
+    if device == "host":
+        if t.is_cuda:
+            raise ValueError(f"{name}: a host tensor is expected")
+    elif device is not None and (not t.is_cuda or t.device.index != device):
+        raise ValueError(f"{name}: expected on cuda:{device}, got {t.device}")
+
+
+def _args(device, *items):
+    """_arg over (tensor, name, numel, kind) items: every dtype and size first, then
+    every device, so a wrong shape is reported before where a tensor lives."""
+    for t, name, numel, kind in items:
+        _arg(t, name, numel, kind, None)
+    for t, name, numel, kind in items:
+        _arg(t, name, numel, kind, device)
+
+
 def _stream(stream):
     if stream is None:
         stream = torch.cuda.current_stream()
@@ -169,9 +201,20 @@ class Plan:
             out = torch.empty((s.batch, s.block, s.q_heads, s.head_dim), dtype=torch.float32, device=q.device)
         if lse is None and want_lse:
             lse = torch.empty((s.batch, s.q_heads, s.block), dtype=torch.float32, device=q.device)
+        nc = s.batch * s.kv_heads * s.ctx_capacity * s.head_dim
+        _args(self.device, *self._decode_items(q, k_blk, v_blk, ctx_lens, out, lse),
+              (k_ctx, "k_ctx", nc, "bf16"), (v_ctx, "v_ctx", nc, "bf16"))
         _check(lib().tt_block_attn(self._h, _ptr(q), _ptr(k_ctx), _ptr(v_ctx), _ptr(k_blk), _ptr(v_blk),
                                    _ptr(ctx_lens), _ptr(out), _ptr(lse), _stream(stream)), "tt_block_attn")
         return (out, lse) if want_lse or lse is not None else out
+
+    def _decode_items(self, q, k_blk, v_blk, ctx_lens, out, lse):
+        s = self.shape
+        nq = s.batch * s.block * s.q_heads * s.head_dim
+        nb = s.batch * s.block * s.kv_heads * s.head_dim
+        return [(q, "q", nq, "bf16"), (k_blk, "k_blk", nb, "bf16"), (v_blk, "v_blk", nb, "bf16"),
+                (ctx_lens, "ctx_lens", s.batch, "i32"), (out, "out", nq, "f32"),
+                (lse, "lse", s.batch * s.q_heads * s.block, "f32")]
 
     def block_attn_paged(self, q, k_pages, v_pages, page_table, k_blk, v_blk, ctx_lens, out=None, lse=None,
                          stream=None, want_lse=False):
@@ -182,8 +225,18 @@ class Plan:
             out = torch.empty((s.batch, s.block, s.q_heads, s.head_dim), dtype=torch.float32, device=q.device)
         if lse is None and want_lse:
             lse = torch.empty((s.batch, s.q_heads, s.block), dtype=torch.float32, device=q.device)
+        if k_pages.dim() != 4 or k_pages.shape[1] != s.kv_heads or k_pages.shape[3] != s.head_dim:
+            raise ValueError(f"k_pages: shape {tuple(k_pages.shape)}, expected [num_pages, {s.kv_heads}, P, "
+                             f"{s.head_dim}]")
         num_pages, _, page_size, _ = k_pages.shape
-        pages_per_seq = page_table.shape[1] if page_table is not None and page_table.dim() == 2 else 0
+        pages_per_seq = 0
+        if page_table is not None:
+            if page_table.dim() != 2 or page_table.shape[0] != s.batch:
+                raise ValueError(f"page_table: shape {tuple(page_table.shape)}, expected [{s.batch}, pages_per_seq]")
+            pages_per_seq = page_table.shape[1]
+        _args(self.device, *self._decode_items(q, k_blk, v_blk, ctx_lens, out, lse),
+              (k_pages, "k_pages", k_pages.numel(), "bf16"), (v_pages, "v_pages", k_pages.numel(), "bf16"),
+              (page_table, "page_table", s.batch * pages_per_seq, "i32"))
         _check(lib().tt_block_attn_paged(self._h, _ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(page_table),
                                          int(num_pages), int(page_size), int(pages_per_seq), _ptr(k_blk),
                                          _ptr(v_blk), _ptr(ctx_lens), _ptr(out), _ptr(lse), _stream(stream)),
@@ -192,6 +245,10 @@ class Plan:
 
     def block_attn_host(self, q, k_ctx, v_ctx, k_blk, v_blk, ctx_lens, out, lse=None, stream=None):
         """Host (ideally pinned) CPU tensors in and out; copies happen inside the library."""
+        s = self.shape
+        nc = s.batch * s.kv_heads * s.ctx_capacity * s.head_dim
+        _args("host", *self._decode_items(q, k_blk, v_blk, ctx_lens, out, lse),
+              (k_ctx, "k_ctx", nc, "bf16"), (v_ctx, "v_ctx", nc, "bf16"))
         _check(lib().tt_block_attn_host(self._h, _ptr(q), _ptr(k_ctx), _ptr(v_ctx), _ptr(k_blk), _ptr(v_blk),
                                         _ptr(ctx_lens), _ptr(out), _ptr(lse), _stream(stream)),
                "tt_block_attn_host")
@@ -205,10 +262,19 @@ class Plan:
             out = torch.empty((s.batch, s.seq_len, s.q_heads, s.head_dim), dtype=torch.float32, device=q.device)
         if lse is None and want_lse:
             lse = torch.empty((s.batch, s.q_heads, s.seq_len), dtype=torch.float32, device=q.device)
+        _args(self.device, *self._causal_items(q, k_ctx, v_ctx, k_blk, v_blk, out, lse))
         _check(lib().tt_block_attn_block_causal(self._h, _ptr(q), _ptr(k_ctx), _ptr(v_ctx), _ptr(k_blk),
                                                 _ptr(v_blk), _ptr(out), _ptr(lse), _stream(stream)),
                "tt_block_attn_block_causal")
         return (out, lse) if want_lse or lse is not None else out
+
+    def _causal_items(self, q, k_ctx, v_ctx, k_blk, v_blk, out, lse):
+        s = self.shape
+        nq = s.batch * s.seq_len * s.q_heads * s.head_dim
+        nk = s.batch * s.seq_len * s.kv_heads * s.head_dim
+        return [(q, "q", nq, "bf16"), (k_ctx, "k_ctx", nk, "bf16"), (v_ctx, "v_ctx", nk, "bf16"),
+                (k_blk, "k_blk", nk, "bf16"), (v_blk, "v_blk", nk, "bf16"), (out, "out", nq, "f32"),
+                (lse, "lse", s.batch * s.q_heads * s.seq_len, "f32")]
 
     def block_causal_backward(self, q, k_ctx, v_ctx, k_blk, v_blk, out, lse, dout, dq=None, dk_blk=None,
                               dv_blk=None, stream=None):
@@ -222,6 +288,11 @@ class Plan:
                                  device=q.device)
         if dv_blk is None:
             dv_blk = torch.empty_like(dk_blk)
+        nq = s.batch * s.seq_len * s.q_heads * s.head_dim
+        nk = s.batch * s.seq_len * s.kv_heads * s.head_dim
+        _args(self.device, *self._causal_items(q, k_ctx, v_ctx, k_blk, v_blk, out, lse),
+              (dout, "dout", nq, "bf16"), (dq, "dq", nq, "f32"), (dk_blk, "dk_blk", nk, "f32"),
+              (dv_blk, "dv_blk", nk, "f32"))
         _check(lib().tt_block_attn_block_causal_backward(
             self._h, _ptr(q), _ptr(k_ctx), _ptr(v_ctx), _ptr(k_blk), _ptr(v_blk), _ptr(out), _ptr(lse), _ptr(dout),
             _ptr(dq), _ptr(dk_blk), _ptr(dv_blk), _stream(stream)), "tt_block_attn_block_causal_backward")
@@ -231,6 +302,11 @@ class Plan:
     def kv_append(self, k_new, v_new, k_ctx, v_ctx, ctx_lens, advance=True, stream=None):
         """Write k_new/v_new [B,S,Hkv,D] into k_ctx/v_ctx [B,Hkv,Lcap,D] at [L_n, L_n+S) in
         place; advance ctx_lens (device int32) by S when `advance`."""
+        s = self.shape
+        nb = s.batch * s.block * s.kv_heads * s.head_dim
+        nc = s.batch * s.kv_heads * s.ctx_capacity * s.head_dim
+        _args(self.device, (k_new, "k_new", nb, "bf16"), (v_new, "v_new", nb, "bf16"), (k_ctx, "k_ctx", nc, "bf16"),
+              (v_ctx, "v_ctx", nc, "bf16"), (ctx_lens, "ctx_lens", s.batch, "i32"))
         _check(lib().tt_kv_append(self._h, _ptr(k_new), _ptr(v_new), _ptr(k_ctx), _ptr(v_ctx), _ptr(ctx_lens),
                                   int(bool(advance)), _stream(stream)), "tt_kv_append")
 
@@ -258,6 +334,9 @@ def confidence_unmask(logits, tokens, masked, gamma=0.8, min_one=True, stream=No
     masked [B,S] uint8 (updated in place).  Returns (p_max [B,S] fp32, argmax [B,S] int32,
     n_committed [B] int32)."""
     B, S, V = logits.shape
+    dev = logits.device.index if logits.device.index is not None else torch.cuda.current_device()
+    _args(dev, (logits, "logits", B * S * V, "bf16"), (tokens, "tokens", B * S, "i32"),
+          (masked, "masked", B * S, "u8"))
     p_max = torch.empty((B, S), dtype=torch.float32, device=logits.device)
     arg = torch.empty((B, S), dtype=torch.int32, device=logits.device)
     n_c = torch.empty((B,), dtype=torch.int32, device=logits.device)
@@ -334,6 +413,11 @@ def block_attn_noalloc(q, k_ctx, v_ctx, k_blk, v_blk, ctx_lens, out, lse=None, s
     `status` is an optional one-element uint32/int32 device tensor for the error bits."""
     B, S, Hq, D = q.shape
     Hkv, Lcap = k_ctx.shape[1], k_ctx.shape[2]
+    dev = q.device.index if q.device.index is not None else torch.cuda.current_device()
+    _args(dev, (q, "q", B * S * Hq * D, "bf16"), (k_ctx, "k_ctx", B * Hkv * Lcap * D, "bf16"),
+          (v_ctx, "v_ctx", B * Hkv * Lcap * D, "bf16"), (k_blk, "k_blk", B * S * Hkv * D, "bf16"),
+          (v_blk, "v_blk", B * S * Hkv * D, "bf16"), (ctx_lens, "ctx_lens", B, "i32"),
+          (out, "out", B * S * Hq * D, "f32"), (lse, "lse", B * Hq * S, "f32"), (status, "status", 1, "w32"))
     d = Desc(B, Hq, Hkv, D, S, Lcap, 0, float(scale), kernel, num_ctas, 0, 0)
     return lib().tt_block_attn_noalloc(ctypes.byref(d), _ptr(q), _ptr(k_ctx), _ptr(v_ctx), _ptr(k_blk),
                                        _ptr(v_blk), _ptr(ctx_lens), _ptr(out), _ptr(lse), _ptr(status),
