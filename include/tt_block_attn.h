@@ -136,10 +136,13 @@ TT_API tt_status_t tt_block_attn(tt_plan_t plan, const void* q, const void* k_ct
                           float* out, float* lse, tt_stream_t stream);
 
 /* Decode over a PAGED context cache: the serving form, where the context tower's
- * layer-i cache of every sequence lives in fixed-size pages drawn from one shared pool
- * (blocks are committed one after another and contexts differ widely in length, so a
- * contiguous Lcap slab per sequence would waste memory).  Same attention as
- * tt_block_attn; only the addressing of the context keys and values differs.
+ * layer-i cache of every sequence lives in fixed-size pages drawn from one shared pool.
+ * The context tower alone holds sequence-length-dependent state, one prefix cache as in
+ * AR serving (paperfeed review of arXiv 2606.26493, "What this changes, and what to be
+ * skeptical of"), and committed blocks are ingested one after another ("Training and
+ * sampling"); with contexts of widely different lengths a contiguous Lcap slab per
+ * sequence would waste memory.  Same attention as tt_block_attn; only the addressing of
+ * the context keys and values differs.
  *   k_pages    [num_pages, Hkv, page_size, D] bf16  key pool (device)
  *   v_pages    [num_pages, Hkv, page_size, D] bf16  value pool (device)
  *   page_table [B, pages_per_seq]             int32 pool page of each sequence's

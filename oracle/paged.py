@@ -3,8 +3,10 @@
 TEST INFRASTRUCTURE ONLY (same rule as ``oracle.oracle``).
 
 Serving keeps each sequence's context-tower cache in fixed-size pages drawn from a
-shared pool (the pages' serving regime: blocks committed and ingested one after the
-other, contexts of very different lengths).  Logical position l of sequence n lives in
+shared pool.  Only the context tower holds sequence-length-dependent state (paperfeed
+review of arXiv 2606.26493, "What this changes, and what to be skeptical of"), and
+committed blocks are ingested one after another ("Training and sampling").  Logical
+position l of sequence n lives in
 page page_table[n, l // P] at offset l % P; the pool is [num_pages, Hkv, P, D].  The
 attention itself is unchanged: gathering the pages back into a contiguous cache and
 calling ``oracle.block_attn`` is the definition.
