@@ -212,3 +212,16 @@ def test_binding_accepts_bf16_bit_patterns_as_two_byte_integers():
     with pytest.raises(TypeError):
         ops._arg(torch.zeros(1, dtype=torch.float32), "status", 1, "w32", None)
     ops._arg(torch.zeros(3), "out", 3, "f32", "host")
+
+
+def test_binding_paged_without_context_needs_no_pool():
+    """No pools and no table: the binding passes NULLs through (valid only without
+    context; the library rejects pages_per_seq > 0 without a pool)."""
+    import torch
+    plan = _shape_only_plan(ctx_capacity=0)
+    B, S, Hq, Hkv, D = 2, 4, 8, 2, 64
+    q = torch.zeros(B, S, Hq, D, dtype=torch.bfloat16)
+    kb = torch.zeros(B, S, Hkv, D, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="q: expected on cuda:0"):    # sizes pass; host memory is refused
+        plan.block_attn_paged(q, None, None, None, kb, kb, torch.zeros(B, dtype=torch.int32),
+                              out=torch.zeros(B, S, Hq, D))

@@ -219,23 +219,28 @@ class Plan:
     def block_attn_paged(self, q, k_pages, v_pages, page_table, k_blk, v_blk, ctx_lens, out=None, lse=None,
                          stream=None, want_lse=False):
         """Decode over a paged context cache: k_pages / v_pages [num_pages, Hkv, P, D] bf16
-        pools, page_table [B, pages_per_seq] int32 (device); P = k_pages.shape[2]."""
+        pools, page_table [B, pages_per_seq] int32 (device); P = k_pages.shape[2].  With no
+        context at all, the pools and the table may be None."""
         s = self.shape
         if out is None:
             out = torch.empty((s.batch, s.block, s.q_heads, s.head_dim), dtype=torch.float32, device=q.device)
         if lse is None and want_lse:
             lse = torch.empty((s.batch, s.q_heads, s.block), dtype=torch.float32, device=q.device)
-        if k_pages.dim() != 4 or k_pages.shape[1] != s.kv_heads or k_pages.shape[3] != s.head_dim:
-            raise ValueError(f"k_pages: shape {tuple(k_pages.shape)}, expected [num_pages, {s.kv_heads}, P, "
-                             f"{s.head_dim}]")
-        num_pages, _, page_size, _ = k_pages.shape
+        if k_pages is None:
+            num_pages, page_size = 0, 16      # no pool: valid only without context (the library checks)
+        else:
+            if k_pages.dim() != 4 or k_pages.shape[1] != s.kv_heads or k_pages.shape[3] != s.head_dim:
+                raise ValueError(f"k_pages: shape {tuple(k_pages.shape)}, expected [num_pages, {s.kv_heads}, P, "
+                                 f"{s.head_dim}]")
+            num_pages, _, page_size, _ = k_pages.shape
+        pool_numel = k_pages.numel() if k_pages is not None else 0
         pages_per_seq = 0
         if page_table is not None:
             if page_table.dim() != 2 or page_table.shape[0] != s.batch:
                 raise ValueError(f"page_table: shape {tuple(page_table.shape)}, expected [{s.batch}, pages_per_seq]")
             pages_per_seq = page_table.shape[1]
         _args(self.device, *self._decode_items(q, k_blk, v_blk, ctx_lens, out, lse),
-              (k_pages, "k_pages", k_pages.numel(), "bf16"), (v_pages, "v_pages", k_pages.numel(), "bf16"),
+              (k_pages, "k_pages", pool_numel, "bf16"), (v_pages, "v_pages", pool_numel, "bf16"),
               (page_table, "page_table", s.batch * pages_per_seq, "i32"))
         _check(lib().tt_block_attn_paged(self._h, _ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(page_table),
                                          int(num_pages), int(page_size), int(pages_per_seq), _ptr(k_blk),
