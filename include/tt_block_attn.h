@@ -156,8 +156,10 @@ TT_API tt_status_t tt_block_attn(tt_plan_t plan, const void* q, const void* k_ct
  * flagged TT_ERR_DEVICE_ARG (as are out-of-range ctx_lens, which are clamped).
  * pages_per_seq == 0 means no context (k_pages / v_pages / page_table may be NULL).
  * Runs the default tcgen05 kernel (whatever TT_TCGEN05_VARIANT selects for
- * tt_block_attn) or the mma.sync kernel, as the plan chose; the caller owns all
- * buffers, nothing is allocated.  TT_ERR_INVALID_ARG for a bad page_size, negative
+ * tt_block_attn) or the mma.sync kernel, as the plan chose, over the plan's work
+ * ranges.  A plan made for the 2-SM form has one range per SM pair, so its paged
+ * calls leave half the SMs idle: make paged plans without that form.  The caller
+ * owns all buffers, nothing is allocated.  TT_ERR_INVALID_ARG for a bad page_size, negative
  * counts, a NULL pointer that is needed or a misaligned one (16 bytes for the bf16
  * and fp32 tensors, 4 for the int32 arrays); TT_ERR_UNSUPPORTED when a pool or a
  * logical capacity holds 2^31 rows or more. */
