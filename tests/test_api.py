@@ -225,3 +225,34 @@ def test_binding_paged_without_context_needs_no_pool():
     with pytest.raises(ValueError, match="q: expected on cuda:0"):    # sizes pass; host memory is refused
         plan.block_attn_paged(q, None, None, None, kb, kb, torch.zeros(B, dtype=torch.int32),
                               out=torch.zeros(B, S, Hq, D))
+
+
+def test_binding_marshals_page_geometry_from_tensor_shapes(monkeypatch):
+    """The paged call hands the library num_pages = pool.shape[0], page_size =
+    pool.shape[2] and pages_per_seq = table.shape[1], in the header's argument order
+    (recorded by a stand-in library; device checks are off for host tensors here)."""
+    import torch
+    seen = {}
+
+    class Rec:
+        def tt_block_attn_paged(self, *a):
+            seen["args"] = a
+            return ops.TT_OK
+
+    monkeypatch.setattr(ops, "lib", lambda: Rec())
+    real_arg = ops._arg
+    monkeypatch.setattr(ops, "_arg", lambda t, n, k, kind, dev: real_arg(t, n, k, kind, None))
+    plan = _shape_only_plan(ctx_capacity=0)
+    B, S, Hq, Hkv, D = 2, 4, 8, 2, 64
+    pool = torch.zeros(7, Hkv, 32, D, dtype=torch.bfloat16)
+    table = torch.zeros(B, 5, dtype=torch.int32)
+    q = torch.zeros(B, S, Hq, D, dtype=torch.bfloat16)
+    kb = torch.zeros(B, S, Hkv, D, dtype=torch.bfloat16)
+    lens = torch.zeros(B, dtype=torch.int32)
+    out = torch.zeros(B, S, Hq, D)
+    monkeypatch.setattr(ops, "_stream", lambda s: None)
+    plan.block_attn_paged(q, pool, pool, table, kb, kb, lens, out=out)
+    a = seen["args"]
+    assert a[5:8] == (7, 32, 5)                                   # num_pages, page_size, pages_per_seq
+    assert a[1].value == q.data_ptr() and a[4].value == table.data_ptr() and a[10].value == lens.data_ptr()
+    assert a[11].value == out.data_ptr() and a[12] is None        # no lse requested
