@@ -1,15 +1,18 @@
 """Benchmark of TwoTower block attention on B200 through the C ABI.
 
-python bench.py [--gpus N] [--steps K] [--warmup W] [--workload ID] [--impl native|reference]
+python bench.py [--gpus N] [--steps K] [--warmup W] [--workload ID] [--only] [--impl native|reference]
 
-One step = one decode call (the whole hot path: Q pack, context KV stream,
-QK^T, online softmax, PV, block-KV fold-in, ragged mask, epilogue, split
-combine) over one batch of the named workload (default: the decode workload
-B=8, Hq=32, Hkv=2, D=128, S=16, L=4096 with 1% peaky keys), or one
-block-causal call for workload 5.  Inputs are resident in HBM before timing;
-each timed step reads a different copy of the inputs and the copies together
-exceed twice the L2 size, so no step is served from L2.  Timing: CUDA events
-on the launching stream around K graph-launched steps, max over ranks.
+One step = one call of the whole hot path (Q pack, context KV stream, QK^T,
+online softmax, PV, block-KV fold-in, ragged mask, epilogue, split combine)
+over one batch of the named workload.  The headline is the long-context
+decode (B=4, Hq=32, Hkv=2, D=128, S=16, L=131072), the largest decode that
+fits one GPU; the line also carries one record per other workload (the
+L=4096 peaky decode, the ragged B=64 decode and the block-causal N=8192
+training form), each timed the same way, unless --only is given.  Inputs are
+resident in HBM before timing; each timed step reads a different copy of the
+inputs and the copies together exceed twice the L2 size, so no step is
+served from L2.  Timing: CUDA events on the launching stream around K
+graph-launched steps, max over ranks.
 
 Prints one JSON line (rank 0).  Multi-GPU runs are replicas: every rank runs
 the same per-GPU batch on its own GPU (weak scaling, no data-path
@@ -42,7 +45,9 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", type=int, default=2, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--workload", type=int, default=4, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--only", action="store_true", help="time the named workload alone (no per-workload records)")
+    ap.add_argument("--no-backward", action="store_true", help="skip the block-causal backward measurement")
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--kernel", default="auto", choices=["auto", "tcgen05", "mma_sync"])
     ap.add_argument("--no-graph", action="store_true", help="launch steps directly instead of via CUDA graphs")
@@ -248,99 +253,217 @@ def run_reference(args):
 
 
 # --------------------------------------------------------------- native arm --
+def roofline_of(wid, cost, k_ms, kname, peaks):
+    """Roofline record of the dominant (attention) kernel of one workload: algorithmic bytes
+    (decode, HBM-bound) or flops (block-causal, tensor-bound) per launch over its average
+    event-timed duration."""
+    from two_tower_block_b200.workloads import WORKLOADS
+    if WORKLOADS[wid].kind == "decode":
+        achieved = cost["bytes"] / (k_ms * 1e-3) / 1e9
+        return {"bound": "hbm", "achieved": round(achieved, 2), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": recorded_traffic(kname, wid),
+                "kernel": f"attn_{kname}", "kernel_ms": round(k_ms, 5),
+                "peak_source": peaks["source"] + " (hbm_gbs, copy)"}
+    ach_t = cost["flops"] / (k_ms * 1e-3) / 1e12
+    pk = peaks["bf16_tflops_sustained"] or peaks["bf16_tflops"]
+    return {"bound": "tensor", "achieved": round(ach_t, 2), "peak": pk, "unit": "TFLOP/s",
+            "frac": round(ach_t / pk, 4), "traffic": recorded_traffic(kname, wid),
+            "kernel": f"attn_{kname}", "kernel_ms": round(k_ms, 5),
+            "peak_source": peaks["source"] + " (bf16_tflops_sustained, cuBLAS)"}
+
+
+class Measured:
+    """One workload resident on the device: its plan, rotating input copies and timings."""
+
+    def __init__(self, wid, args, dev, kernel, local):
+        import torch
+        from two_tower_block_b200 import ops
+        from two_tower_block_b200.workloads import WORKLOADS, make_workload
+        self.wid, self.w = wid, WORKLOADS[wid]
+        w = self.w
+        self.inp = make_workload(wid)
+        self.cost = workload_cost(wid, self.inp)
+        self.l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+
+        def to_dev(bits):
+            return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+        self.to_dev = to_dev
+        base = [to_dev(self.inp.q), to_dev(self.inp.k_ctx), to_dev(self.inp.v_ctx), to_dev(self.inp.k_blk),
+                to_dev(self.inp.v_blk)]
+        self.in_bytes = sum(t.numel() * 2 for t in base)
+        self.n_copies = max(1, math.ceil(2.0 * self.l2 / self.in_bytes) + 1)
+        self.copies = [base] + [[t.clone() for t in base] for _ in range(self.n_copies - 1)]
+        if w.kind == "decode":
+            self.lens = torch.from_numpy(self.inp.ctx_lens).to(dev)
+            self.plan = ops.Plan(w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_size,
+                                 ctx_capacity=w.ctx, kernel=kernel, num_ctas=args.num_ctas, device=local)
+            self.out = torch.empty((w.batch, w.block_size, w.num_q_heads, w.head_dim), dtype=torch.float32,
+                                   device=dev)
+            self.lse = torch.empty((w.batch, w.num_q_heads, w.block_size), dtype=torch.float32, device=dev)
+        else:
+            self.lens = None
+            self.plan = ops.Plan(w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_size,
+                                 seq_len=w.seq_len, kernel=kernel, num_ctas=args.num_ctas, device=local)
+            self.out = torch.empty((w.batch, w.seq_len, w.num_q_heads, w.head_dim), dtype=torch.float32,
+                                   device=dev)
+            self.lse = torch.empty((w.batch, w.num_q_heads, w.seq_len), dtype=torch.float32, device=dev)
+        self.info = self.plan.info()
+        kname = {1: "tcgen05", 2: "mma_sync"}[self.info.kernel]
+        if self.info.kernel == 1 and self.info.variant in (2, 3):   # the selectable forms have their own sources
+            kname = {2: "tcgen05_pt", 3: "tcgen05_2sm"}[self.info.variant]
+        self.kname = kname
+
+    def step(self, i):
+        c = self.copies[i % self.n_copies]
+        if self.w.kind == "decode":
+            self.plan.block_attn(c[0], c[1], c[2], c[3], c[4], self.lens, out=self.out, lse=self.lse)
+        else:
+            self.plan.block_attn_block_causal(c[0], c[1], c[2], c[3], c[4], out=self.out, lse=self.lse)
+
+    def time(self, args, pg, dev, before_timed=None):
+        """W warm-up steps, then K timed steps (graph replay unless --no-graph) between a barrier and a
+        synchronize on both sides; then the same K steps again with the library's per-kernel events."""
+        import torch
+        stream = torch.cuda.current_stream()
+        for i in range(max(3, args.warmup)):
+            self.step(i)
+        self.plan.check()
+        graphs = None
+        if not args.no_graph:
+            graphs = []
+            for i in range(self.n_copies):
+                gph = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(gph):
+                    self.step(i)
+                graphs.append(gph)
+            for g in graphs:
+                g.replay()
+            torch.cuda.synchronize()
+        if before_timed:
+            before_timed()
+        if pg:
+            pg.barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(args.steps):
+            if graphs:
+                graphs[i % self.n_copies].replay()
+            else:
+                self.step(i)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if pg:
+            pg.barrier()
+        ms_total = e0.elapsed_time(e1)
+        # per-kernel durations of the same steps, from events the library records on the launching stream
+        self.plan.profile(True)
+        for i in range(args.steps):
+            self.step(i)
+        torch.cuda.synchronize()
+        n_k, ms_k = self.plan.profile_read(0)
+        n_c, ms_c = self.plan.profile_read(1) if self.info.num_ctas > 1 else (0, 0.0)
+        self.plan.profile(False)
+        self.plan.check()
+        del graphs
+        self.ms_step = max_over_ranks(pg, ms_total, dev) / args.steps
+        self.k_ms = ms_k / max(n_k, 1)
+        self.c_ms = ms_c / max(n_c, 1) if n_c else None
+        self.launches_per_step = (n_k + n_c) // max(args.steps, 1)
+        self.graphs_used = graphs is not None or not args.no_graph
+
+    def record(self, world, peaks):
+        value = replica_rate(world, self.cost["bytes"], self.ms_step) / 1e9
+        tflops = replica_rate(world, self.cost["flops"], self.ms_step) / 1e12
+        return {"workload": self.w.name, "value": round(value, 3), "unit": "GB/s",
+                "ms_per_step": round(self.ms_step, 5), "tflops": round(tflops, 2),
+                "alg_bytes": int(self.cost["bytes"]), "flops": int(self.cost["flops"]),
+                "roofline": roofline_of(self.wid, self.cost, self.k_ms, self.kname, peaks),
+                "combine_kernel_ms": round(self.c_ms, 5) if self.c_ms else None,
+                "launches_per_step": self.launches_per_step, "num_ctas": self.info.num_ctas,
+                "l2": "inputs rotate over %d copies (%.0f MB) > 2x L2 (%d MB)" % (
+                    self.n_copies, self.n_copies * self.in_bytes / 1e6, self.l2 // 2**20)}
+
+    def free(self):
+        self.plan.close()
+        del self.copies, self.out, self.lse
+
+
+def measure_backward(m, dev):
+    """Block-causal backward at a training workload's shape: device time of its kernel."""
+    import torch
+    w, plan, c0 = m.w, m.plan, m.copies[0]
+    bout = torch.empty((w.batch, w.seq_len, w.num_q_heads, w.head_dim), dtype=torch.float32, device=dev)
+    blse = torch.empty((w.batch, w.num_q_heads, w.seq_len), dtype=torch.float32, device=dev)
+    plan.block_attn_block_causal(c0[0], c0[1], c0[2], c0[3], c0[4], out=bout, lse=blse)
+    dout = torch.empty_like(bout).normal_().to(torch.bfloat16)
+    dq = torch.empty_like(bout)
+    dkb = torch.empty((w.batch, w.seq_len, w.num_kv_heads, w.head_dim), dtype=torch.float32, device=dev)
+    dvb = torch.empty_like(dkb)
+    for _ in range(2):
+        plan.block_causal_backward(c0[0], c0[1], c0[2], c0[3], c0[4], bout, blse, dout, dq, dkb, dvb)
+    torch.cuda.synchronize()
+    plan.profile(True)
+    n_b = 3
+    for _ in range(n_b):
+        plan.block_causal_backward(c0[0], c0[1], c0[2], c0[3], c0[4], bout, blse, dout, dq, dkb, dvb)
+    torch.cuda.synchronize()
+    nb_l, ms_b = plan.profile_read(2)
+    plan.profile(False)
+    plan.check()
+    ms_b /= max(nb_l, 1)
+    # recompute S, dP and dQ over every visible key (3 x 2D flops per row and key),
+    # dK and dV over the block's own keys (2 x 2D per row and block key)
+    rows_keys = m.cost["flops"] / (4 * w.head_dim)
+    rows_blk = w.batch * w.num_q_heads * w.seq_len * w.block_size
+    bflops = 6 * w.head_dim * rows_keys + 4 * w.head_dim * rows_blk
+    pkk = load_peaks()
+    pk = pkk["bf16_tflops_sustained"] or pkk["bf16_tflops"]
+    del bout, blse, dout, dq, dkb, dvb
+    return {"kernel": "attn_bwd", "ms": round(ms_b, 4), "tflops": round(bflops / (ms_b * 1e-3) / 1e12, 2),
+            "frac_of_sustained_bf16": round(bflops / (ms_b * 1e-3) / 1e12 / pk, 4), "launches": nb_l}
+
+
 def run_native(args):
     import torch
     world, rank, local, pg = dist_setup(args)
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     from two_tower_block_b200 import ops
-    from two_tower_block_b200.workloads import WORKLOADS, make_workload
-    w = WORKLOADS[args.workload]
     kernel = {"auto": ops.KERNEL_AUTO, "tcgen05": ops.KERNEL_TCGEN05, "mma_sync": ops.KERNEL_MMA_SYNC}[args.kernel]
-    inp = make_workload(args.workload)
-    cost = workload_cost(args.workload, inp)
-    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-
-    def to_dev(bits):
-        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
-
-    base = [to_dev(inp.q), to_dev(inp.k_ctx), to_dev(inp.v_ctx), to_dev(inp.k_blk), to_dev(inp.v_blk)]
-    in_bytes = sum(t.numel() * 2 for t in base)
-    n_copies = max(1, math.ceil(2.0 * l2 / in_bytes) + 1)
-    copies = [base] + [[t.clone() for t in base] for _ in range(n_copies - 1)]
-    if w.kind == "decode":
-        lens = torch.from_numpy(inp.ctx_lens).to(dev)
-        plan = ops.Plan(w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_size, ctx_capacity=w.ctx,
-                        kernel=kernel, num_ctas=args.num_ctas, device=local)
-        out = torch.empty((w.batch, w.block_size, w.num_q_heads, w.head_dim), dtype=torch.float32, device=dev)
-        lse = torch.empty((w.batch, w.num_q_heads, w.block_size), dtype=torch.float32, device=dev)
-
-        def step(i):
-            c = copies[i % n_copies]
-            plan.block_attn(c[0], c[1], c[2], c[3], c[4], lens, out=out, lse=lse)
-    else:
-        plan = ops.Plan(w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_size, seq_len=w.seq_len,
-                        kernel=kernel, num_ctas=args.num_ctas, device=local)
-        out = torch.empty((w.batch, w.seq_len, w.num_q_heads, w.head_dim), dtype=torch.float32, device=dev)
-        lse = torch.empty((w.batch, w.num_q_heads, w.seq_len), dtype=torch.float32, device=dev)
-
-        def step(i):
-            c = copies[i % n_copies]
-            plan.block_attn_block_causal(c[0], c[1], c[2], c[3], c[4], out=out, lse=lse)
-
-    info = plan.info()
-    kname = {1: "tcgen05", 2: "mma_sync"}[info.kernel]
-    if info.kernel == 1 and info.variant in (2, 3):   # the selectable tcgen05 forms have their own sources
-        kname = {2: "tcgen05_pt", 3: "tcgen05_2sm"}[info.variant]
-    stream = torch.cuda.current_stream()
-    for i in range(max(3, args.warmup)):
-        step(i)
-    plan.check()
-
-    graphs = None
-    if not args.no_graph:
-        graphs = []
-        for i in range(n_copies):
-            gph = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(gph):
-                step(i)
-            graphs.append(gph)
-        for i in range(n_copies):
-            graphs[i].replay()
-        torch.cuda.synchronize()
+    peaks = load_peaks()
 
     clocks = ClockSampler(local)
-    if pg:
-        pg.barrier()
-    torch.cuda.synchronize()
-    clocks.start()
-    time.sleep(0.3)  # let the sampler attach before the timed region
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for i in range(args.steps):
-        if graphs:
-            graphs[i % n_copies].replay()
-        else:
-            step(i)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    if pg:
-        pg.barrier()
-    ms_total = e0.elapsed_time(e1)
-    # per-kernel durations of the same steps, from events the library records on the launching stream
-    plan.profile(True)
-    for i in range(args.steps):
-        step(i)
-    torch.cuda.synchronize()
-    n_k, ms_k = plan.profile_read(0)
-    n_c, ms_c = plan.profile_read(1) if info.num_ctas > 1 else (0, 0.0)
-    plan.profile(False)
+    started = []
+
+    def start_clocks():
+        if not started:
+            clocks.start()
+            time.sleep(0.3)  # let the sampler attach before the first timed region
+            started.append(1)
+
+    # the other workloads first, each timed the same way and freed before the next
+    extra = []
+    extra_ids = [] if args.only else [x for x in (2, 3, 4, 5) if x != args.workload]
+    bwd = None
+    for wid in extra_ids:
+        m = Measured(wid, args, dev, kernel, local)
+        m.time(args, pg, dev, before_timed=start_clocks)
+        extra.append(m.record(world, peaks))
+        if m.w.kind == "causal" and not args.no_backward:
+            bwd = measure_backward(m, dev)
+            extra[-1]["backward"] = bwd
+        m.free()
+        del m
+        torch.cuda.empty_cache()
+
+    m = Measured(args.workload, args, dev, kernel, local)
+    w, inp, cost, plan, info = m.w, m.inp, m.cost, m.plan, m.info
+    m.time(args, pg, dev, before_timed=start_clocks)
     ck = clocks.stop()
-    plan.check()
-    ms_total = max_over_ranks(pg, ms_total, dev)
-    ms_step = ms_total / args.steps
-    # one attention launch per step, plus the split combine when it ran as its own kernel
-    launches_per_step = 1 + (1 if n_c > 0 else 0)
+    stream = torch.cuda.current_stream()
+    ms_step = m.ms_step
+    out, lse = m.out, m.lse
 
     # ---- end to end through the host-buffer entry (decode workloads) ----
     e2e = None
@@ -371,6 +494,8 @@ def run_native(args):
         e2e = {"value": round(world * cost["bytes"] / (ms_e2e * 1e-3) / 1e9, 3), "unit": "GB/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": round(ms_e2e, 4),
                "steps": n_e2e}
+        hplan.close()
+        del hin, hout, hlse
 
     # ---- the same decode over a paged cache: pages of --page-size rows in a shuffled pool ----
     paged = None
@@ -379,21 +504,22 @@ def run_native(args):
         P = args.page_size
         pc = make_paged(inp, P, seed=w.seed, spare_pages=0, fill_bits=0)
         ptab = torch.from_numpy(pc.page_table).to(dev)
-        pbase = [to_dev(pc.k_pages), to_dev(pc.v_pages)]
-        pcopies = [pbase] + [[t.clone() for t in pbase] for _ in range(n_copies - 1)]
+        pbase = [m.to_dev(pc.k_pages), m.to_dev(pc.v_pages)]
+        del pc
+        pcopies = [pbase] + [[t.clone() for t in pbase] for _ in range(m.n_copies - 1)]
         pplan = ops.Plan(w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_size, ctx_capacity=0,
                          kernel=kernel, num_ctas=args.num_ctas, device=local)
 
         def pstep(i):
-            c, pk = copies[i % n_copies], pcopies[i % n_copies]
-            pplan.block_attn_paged(c[0], pk[0], pk[1], ptab, c[3], c[4], lens, out=out, lse=lse)
+            c, pk = m.copies[i % m.n_copies], pcopies[i % m.n_copies]
+            pplan.block_attn_paged(c[0], pk[0], pk[1], ptab, c[3], c[4], m.lens, out=out, lse=lse)
         for i in range(max(3, args.warmup)):
             pstep(i)
         pplan.check()
         pgraphs = None
         if not args.no_graph:
             pgraphs = []
-            for i in range(n_copies):
+            for i in range(m.n_copies):
                 gph = torch.cuda.CUDAGraph()
                 with torch.cuda.graph(gph):
                     pstep(i)
@@ -405,7 +531,7 @@ def run_native(args):
         p0.record(stream)
         for i in range(args.steps):
             if pgraphs:
-                pgraphs[i % n_copies].replay()
+                pgraphs[i % m.n_copies].replay()
             else:
                 pstep(i)
         p1.record(stream)
@@ -422,45 +548,16 @@ def run_native(args):
         pk_ms = ms_pk / max(n_pk, 1)
         tbytes = int(sum(-(-int(L) // P) for L in inp.ctx_lens)) * 4 * w.num_kv_heads   # table entries read
         pbytes = cost["bytes"] + tbytes
-        paged = {"page_size": P, "pool_pages": int(pc.k_pages.shape[0]), "ms_per_step": round(ms_pstep, 5),
+        paged = {"page_size": P, "pool_pages": int(pbase[0].shape[0]), "ms_per_step": round(ms_pstep, 5),
                  "value": round(replica_rate(world, pbytes, ms_pstep) / 1e9, 3), "unit": "GB/s",
                  "kernel_ms": round(pk_ms, 5), "kernel_gbs": round(pbytes / (pk_ms * 1e-3) / 1e9, 2),
-                 "kernel_time_vs_contiguous": round(pk_ms / (ms_k / max(n_k, 1)), 4),
+                 "kernel_time_vs_contiguous": round(pk_ms / m.k_ms, 4),
                  "launches_per_step": (n_pk + n_pc) // max(args.steps, 1)}
-        del pcopies, pbase
+        del pgraphs, pcopies, pbase
+        pplan.close()
 
-    # ---- block-causal backward at this workload's shape (training workloads) ----
-    bwd = None
-    if w.kind == "causal":
-        c0 = copies[0]
-        bout = torch.empty((w.batch, w.seq_len, w.num_q_heads, w.head_dim), dtype=torch.float32, device=dev)
-        blse = torch.empty((w.batch, w.num_q_heads, w.seq_len), dtype=torch.float32, device=dev)
-        plan.block_attn_block_causal(c0[0], c0[1], c0[2], c0[3], c0[4], out=bout, lse=blse)
-        dout = torch.empty_like(bout).normal_().to(torch.bfloat16)
-        dq = torch.empty_like(bout)
-        dkb = torch.empty((w.batch, w.seq_len, w.num_kv_heads, w.head_dim), dtype=torch.float32, device=dev)
-        dvb = torch.empty_like(dkb)
-        for _ in range(2):
-            plan.block_causal_backward(c0[0], c0[1], c0[2], c0[3], c0[4], bout, blse, dout, dq, dkb, dvb)
-        torch.cuda.synchronize()
-        plan.profile(True)
-        n_b = 3
-        for _ in range(n_b):
-            plan.block_causal_backward(c0[0], c0[1], c0[2], c0[3], c0[4], bout, blse, dout, dq, dkb, dvb)
-        torch.cuda.synchronize()
-        nb_l, ms_b = plan.profile_read(2)
-        plan.profile(False)
-        plan.check()
-        ms_b /= max(nb_l, 1)
-        # recompute S, dP and dQ over every visible key (3 x 2D flops per row and key),
-        # dK and dV over the block's own keys (2 x 2D per row and block key)
-        rows_keys = cost["flops"] / (4 * w.head_dim)
-        rows_blk = w.batch * w.num_q_heads * w.seq_len * w.block_size
-        bflops = 6 * w.head_dim * rows_keys + 4 * w.head_dim * rows_blk
-        pkk = load_peaks()
-        pk = pkk["bf16_tflops_sustained"] or pkk["bf16_tflops"]
-        bwd = {"kernel": "attn_bwd (mma.sync)", "ms": round(ms_b, 4), "tflops": round(bflops / (ms_b * 1e-3) / 1e12, 2),
-               "frac_of_sustained_bf16": round(bflops / (ms_b * 1e-3) / 1e12 / pk, 4), "launches": nb_l}
+    if w.kind == "causal" and not args.no_backward:
+        bwd = measure_backward(m, dev)
 
     # ---- committed-block cache update at this workload's shape (decode only) ----
     kv_app = None
@@ -492,14 +589,17 @@ def run_native(args):
         nbytes = 4 * B_ * S_ * H_ * D_ * 2       # K and V: read the new rows, write them into the cache
         kv_app = {"us_per_call": round(us, 3), "bytes": nbytes, "gbs": round(nbytes / (us * 1e-6) / 1e9, 2),
                   "launches": n_app}
+        del ag
+        aplan.close()
 
     # ---- confidence-unmasking step over a 131072-entry vocabulary at the block shape ----
     unmask = None
     if w.kind == "decode":
         Vv = 131072
-        lg = torch.empty((w.batch, w.block_size, Vv), dtype=torch.bfloat16, device=dev).normal_()
-        tk = torch.full((w.batch, w.block_size), -1, dtype=torch.int32, device=dev)
-        mk = torch.ones((w.batch, w.block_size), dtype=torch.uint8, device=dev)
+        UB = 8   # eight sequences of S block positions (the decode batch of the L = 4096 workload)
+        lg = torch.empty((UB, w.block_size, Vv), dtype=torch.bfloat16, device=dev).normal_()
+        tk = torch.full((UB, w.block_size), -1, dtype=torch.int32, device=dev)
+        mk = torch.ones((UB, w.block_size), dtype=torch.uint8, device=dev)
         # standard-normal logits never reach 0.8 and min_one is off: every call scans every row
         for _ in range(3):
             ops.confidence_unmask(lg, tk, mk, gamma=0.8, min_one=False)
@@ -516,9 +616,11 @@ def run_native(args):
         u1.record(stream)
         torch.cuda.synchronize()
         us = u0.elapsed_time(u1) * 1e3 / n_u
-        ubytes = w.batch * w.block_size * Vv * 2
-        unmask = {"vocab": Vv, "us_per_call": round(us, 3), "bytes": ubytes,
-                  "gbs": round(ubytes / (us * 1e-6) / 1e9, 2), "launches_per_call": 2}
+        ubytes = UB * w.block_size * Vv * 2
+        unmask = {"rows": UB * w.block_size, "vocab": Vv, "us_per_call": round(us, 3), "bytes": ubytes,
+                  "gbs": round(ubytes / (us * 1e-6) / 1e9, 2),
+                  "frac_hbm": round(ubytes / (us * 1e-6) / 1e9 / peaks["hbm_gbs"], 4), "launches_per_call": 2}
+        del ug, lg
 
     # ---- oracle CPU baseline (rank 0, N = 1 only) ----
     cpu = None
@@ -528,41 +630,24 @@ def run_native(args):
                "sample": desc + f"; host has {os.cpu_count()} logical CPUs"}
 
     if rank != 0:
+        m.free()
         return 0
-    peaks = load_peaks()
-    value = replica_rate(world, cost["bytes"], ms_step) / 1e9      # ms_step is already the max over ranks
-    tflops = replica_rate(world, cost["flops"], ms_step) / 1e12
-    k_ms = ms_k / max(n_k, 1)
-    achieved = cost["bytes"] / (k_ms * 1e-3) / 1e9
-    bound = "hbm" if w.kind == "decode" else "tensor"
-    if bound == "hbm":
-        roof = {"bound": "hbm", "achieved": round(achieved, 2), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": recorded_traffic(kname, args.workload),
-                "kernel": f"attn_{kname}", "kernel_ms": round(k_ms, 5),
-                "peak_source": peaks["source"] + " (hbm_gbs, copy)"}
-    else:
-        ach_t = cost["flops"] / (k_ms * 1e-3) / 1e12
-        pk = peaks["bf16_tflops_sustained"] or peaks["bf16_tflops"]
-        roof = {"bound": "tensor", "achieved": round(ach_t, 2), "peak": pk, "unit": "TFLOP/s",
-                "frac": round(ach_t / pk, 4), "traffic": recorded_traffic(kname, args.workload),
-                "kernel": f"attn_{kname}", "kernel_ms": round(k_ms, 5),
-                "peak_source": peaks["source"] + " (bf16_tflops_sustained, cuBLAS)"}
+    rec = m.record(world, peaks)
     line = {
-        "metric": METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True, "scaling": "weak",
+        "metric": METRIC, "value": rec["value"], "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": rec["ms_per_step"], "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": dict(w.describe(), parallelism=f"replicas{world}",
-                       l2="inputs rotate over %d copies (%.0f MB) > 2x L2 (%d MB)" % (
-                           n_copies, n_copies * in_bytes / 1e6, l2 // 2**20),
-                       timing="graph replay" if graphs else "direct launches"),
-        "tflops": round(tflops, 2),
-        "tensor_frac": round(tflops / peaks["bf16_tflops"], 4),
-        "roofline": roof,
-        "combine_kernel_ms": round(ms_c / max(n_c, 1), 5) if n_c else None,
-        "gpu_launches": launches_per_step * args.steps,
-        "kernel": kname,
+        "config": dict(w.describe(), parallelism=f"replicas{world}", l2=rec["l2"],
+                       timing="graph replay" if not args.no_graph else "direct launches"),
+        "tflops": rec["tflops"],
+        "tensor_frac": round(rec["tflops"] / peaks["bf16_tflops"], 4),
+        "roofline": rec["roofline"],
+        "combine_kernel_ms": rec["combine_kernel_ms"],
+        "gpu_launches": m.launches_per_step * args.steps,
+        "kernel": m.kname,
         "num_ctas": info.num_ctas,
         "e2e": e2e,
+        "workloads": extra,
         "kv_append": kv_app,
         "paged": paged,
         "backward": bwd,
@@ -570,6 +655,7 @@ def run_native(args):
         "cpu_baseline": cpu,
         "clocks": ck,
     }
+    m.free()
     print(json.dumps(line), flush=True)
     if pg:
         pg.destroy_process_group()

@@ -9,7 +9,7 @@
  * frozen context tower's layer-i KV cache over every committed token,
  * followed by the denoiser's own KV for the block.  The cache is fully
  * visible (only the context tower itself is causal), attention inside the
- * block is bidirectional ("masked tokens can look at each other"), and one
+ * block is bidirectional, still-masked positions included, and one
  * softmax runs over the concatenation.  The page's equation was lost in
  * extraction; the single joint softmax is the reading of its prose.
  *
@@ -255,7 +255,7 @@ TT_API tt_status_t tt_confidence_unmask(const void* logits, int batch, int block
 
 /* Committed-block cache update (paperfeed.app review of arXiv 2606.26493, section
  * "The idea: freeze the reader, train the writer": a committed block is ingested by
- * the frozen context tower, "updating its caches").  For every sequence n:
+ * the frozen context tower, which extends its per-layer caches).  For every sequence n:
  *   k_ctx[n, h, L_n + t, :] = k_new[n, t, h, :],  v_ctx likewise,  t < S, h < Hkv,
  * with L_n = ctx_lens[n] read on the device, and then, when `advance` is non-zero,
  * ctx_lens[n] = L_n + S.

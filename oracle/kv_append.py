@@ -6,7 +6,7 @@ TEST INFRASTRUCTURE ONLY (same rule as ``oracle.oracle``): only ``tests/``,
 What it computes (paperfeed.app review of arXiv 2606.26493, section "The idea:
 freeze the reader, train the writer", last paragraphs): once every token of a
 block is resolved the block is committed and the frozen context tower ingests
-it causally, "updating its caches".  The context tower's layer-i keys and
+it causally, which extends its per-layer caches.  The context tower's layer-i keys and
 values of the S committed positions (computed by the caller) are written into
 the cache right after the L_n tokens already committed, and the committed
 length grows by S.  Plain reading of a step the page states only in words:

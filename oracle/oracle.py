@@ -16,11 +16,11 @@ attention; and section "Training and sampling" for the block-causal form):
 * the denoiser's queries come from the S noisy tokens of the current block;
 * the keys and values are the concatenation of the frozen context tower's
   layer-i KV cache over the committed tokens with the denoiser's own KV for
-  the block ("the keys/values concatenate ... cache for past blocks with the
-  denoiser's own KV for the current block");
+  the block (same section: the page describes the denoiser's layer-i keys and
+  values as the context cache of the earlier blocks joined to the block's own);
 * the cache is fully visible to every block query (only the context tower
-  itself is causal), and attention inside the block is bidirectional
-  ("masked tokens can look at each other");
+  itself is causal), and attention inside the block is bidirectional, still-masked
+  positions included (same section, on the block's own attention);
 * one softmax runs over the concatenation.  The equation itself did not
   survive the page extraction; the joint softmax is the plain reading of the
   surrounding prose.

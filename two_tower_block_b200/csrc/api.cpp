@@ -97,6 +97,7 @@ struct tt_plan_s {
   unsigned* err_word = nullptr;
   unsigned long long* grid_bar = nullptr;  // fused combine's grid barrier (in the error-word block)
   bool fused_combine = false;
+  bool pingpong = false;
   int* causal_pref = nullptr;
   long long causal_T = 0;
   int causal_NB = 0;
@@ -159,6 +160,7 @@ tt::Problem base_problem(tt_plan_t plan) {
   p.wait_limit_ns = (unsigned long long)(d.wait_timeout_us > 0 ? d.wait_timeout_us : 1000000) * 1000ull;
   p.variant = plan->variant;
   p.grid_bar = plan->fused_combine ? plan->grid_bar : nullptr;
+  p.pingpong = plan->pingpong ? 1 : 0;
   return p;
 }
 
@@ -296,6 +298,9 @@ tt_status_t tt_block_attn_plan(const tt_block_attn_desc* desc, int device, tt_pl
       const int v = std::atoi(kv);
       P->variant = (v == 2 || v == 3) ? v : 0;
     }
+    // TT_PINGPONG=1: the two softmax warpgroups of the default kernel take turns at the
+    // exponentials (measured slower on the decode workloads, so off by default)
+    if (const char* pp = std::getenv("TT_PINGPONG")) P->pingpong = std::atoi(pp) != 0;
     if (P->variant == 3 && (!tt::attn_2sm_supported(d.head_dim, g) || P->key_tile != 128)) P->variant = 0;
     P->C = d.num_ctas > 0 ? d.num_ctas : P->sm_count;
     if (P->variant == 3) {

@@ -27,6 +27,13 @@
 // buffer PV(j) has just consumed; with two buffers the softmax of tile j+1
 // finds its S ready while the tensor core works on PV(j).
 //
+// Ping-pong: with two M-tiles the softmax warpgroups take turns at the
+// exponentials (tile G of warpgroup 1 after tile G of warpgroup 0, tile G+1 of
+// warpgroup 0 after that).  Without it both warpgroups receive their scores at
+// the same moment, share the MUFU for the whole tile and leave the tensor core
+// idle meanwhile; with it one M-tile's PV and next S run on the tensor core
+// while the other M-tile's softmax runs.
+//
 // The softmax keeps a running reference maximum per row and rescales O (in
 // TMEM) only when a new maximum exceeds it by more than 2^8; the final
 // normalisation divides by the sum of the same bf16-rounded weights the PV
@@ -72,6 +79,7 @@ struct Bars {
   uint64_t q_full, q_empty, tail, drain;
   uint64_t s_full[2][2], p_full[2][2];  // [M-tile][S buffer]
   uint64_t pv_done[2], o_full[2], o_empty[2];
+  uint64_t turn[2];                     // ping-pong: warpgroup m may start its exponentials
   uint64_t kv_full[16], kv_empty[16];
 };
 
@@ -81,6 +89,7 @@ struct Shared {
   long long T, start, end;
   Unit first;
 };
+static_assert(sizeof(Bars) + sizeof(Shared) <= 512, "barrier block overflows its shared-memory slot");
 
 // Fused split combine (cooperative launch only): every CTA arrives at a grid barrier once
 // its segments and its split record are written, then the CTAs share the rows of the cut
@@ -179,6 +188,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(smem_u32(&bars->pv_done[m]), 1);
       mbar_init(smem_u32(&bars->o_full[m]), 1);
       mbar_init(smem_u32(&bars->o_empty[m]), 128);
+      mbar_init(smem_u32(&bars->turn[m]), 4);  // one arrival per warp of the other warpgroup
     }
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(smem_u32(&bars->kv_full[s]), 1);
@@ -405,6 +415,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = q4 * 32 + lane;      // row within the M-tile
     const int r = m * 128 + row;         // packed row of the unit
     if (m < MT) {
+      const bool pp = MT == 2 && p.pingpong != 0;
+      const uint32_t turn_mine = smem_u32(&bars->turn[m]), turn_other = smem_u32(&bars->turn[m ^ 1]);
       const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
       const uint32_t s_base = tmem + lane_off + m * 128;  // + buffer * NK
       const uint32_t o_addr = tmem + lane_off + 256 + m * D;
@@ -455,8 +467,19 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
             }
           }
+          // ping-pong turn: warpgroup 0 runs the exponentials of its tile G once warpgroup 1
+          // finished those of tile G-1 (completion G-1 of turn[0]); warpgroup 1 those of tile G
+          // once warpgroup 0 finished tile G (completion G of turn[1]).  Warpgroup 0 starts.
+          if (pp && (m == 1 || G > 0)) {
+            ok = mbar_wait(turn_mine, (m == 0 ? G - 1 : G) & 1, wc);
+            if (!ok) break;
+          }
           l += full ? tile_exp_store<NK, true>(v, count, p.scale_log2, m_ref, s_addr)
                     : tile_exp_store<NK, false>(v, count, p.scale_log2, m_ref, s_addr);
+          if (pp) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(turn_other);
+          }
           tc_wait_st();
           tc_fence_before();
           mbar_arrive(smem_u32(&bars->p_full[m][b]));

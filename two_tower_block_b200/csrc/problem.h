@@ -47,6 +47,8 @@ struct Problem {
   unsigned long long wait_limit_ns;
   int variant;          // tcgen05 kernel: 0 = S/P aliasing in TMEM (default), 2 = transposed PV,
                         // 3 = 2-SM pairs (head_dim 128)
+  int pingpong;         // default tcgen05 kernel with two M-tiles: the softmax warpgroups take turns
+                        // at the exponentials, so one M-tile's MMAs run during the other's softmax
   // default tcgen05 kernel launched cooperatively: the CTAs meet at this grid barrier
   // (a counter that only grows) and combine the cut units themselves; null: the
   // separate combine kernel runs instead
