@@ -97,7 +97,6 @@ struct tt_plan_s {
   unsigned* err_word = nullptr;
   unsigned long long* grid_bar = nullptr;  // fused combine's grid barrier (in the error-word block)
   bool fused_combine = false;
-  bool pingpong = false;
   int* causal_pref = nullptr;
   long long causal_T = 0;
   int causal_NB = 0;
@@ -160,7 +159,6 @@ tt::Problem base_problem(tt_plan_t plan) {
   p.wait_limit_ns = (unsigned long long)(d.wait_timeout_us > 0 ? d.wait_timeout_us : 1000000) * 1000ull;
   p.variant = plan->variant;
   p.grid_bar = plan->fused_combine ? plan->grid_bar : nullptr;
-  p.pingpong = plan->pingpong ? 1 : 0;
   return p;
 }
 
@@ -287,20 +285,19 @@ tt_status_t tt_block_attn_plan(const tt_block_attn_desc* desc, int device, tt_pl
   if (P->kernel == TT_KERNEL_TCGEN05 && prop.major != 10) P->kernel = TT_KERNEL_MMA_SYNC;
   if (P->kernel == TT_KERNEL_TCGEN05) {
     P->key_tile = tt::kTcgen05KeyTile;
-    // tuning knobs: TT_TCGEN05_KEY_TILE=64 selects the two-buffer 64-key pipeline;
+    // tuning knobs: TT_TCGEN05_KEY_TILE=128 selects the one-buffer 128-key pipeline;
     // TT_TCGEN05_VARIANT=2 selects the transposed-PV kernel for head_dim 128,
-    // TT_TCGEN05_VARIANT=3 the 2-SM kernel (head_dim 128, 128 % g == 0)
+    // TT_TCGEN05_VARIANT=3 the 2-SM kernel (head_dim 128, 128 % g == 0); both run 128-key
+    // tiles, which they select unless a key tile is given
+    if (const char* kv = std::getenv("TT_TCGEN05_VARIANT")) {
+      const int v = std::atoi(kv);
+      P->variant = (v == 2 || v == 3) ? v : 0;
+      if (P->variant != 0) P->key_tile = 128;
+    }
     if (const char* kt = std::getenv("TT_TCGEN05_KEY_TILE")) {
       const int v = std::atoi(kt);
       if (tt::tcgen05_key_tile_supported(v)) P->key_tile = v;
     }
-    if (const char* kv = std::getenv("TT_TCGEN05_VARIANT")) {
-      const int v = std::atoi(kv);
-      P->variant = (v == 2 || v == 3) ? v : 0;
-    }
-    // TT_PINGPONG=1: the two softmax warpgroups of the default kernel take turns at the
-    // exponentials (measured slower on the decode workloads, so off by default)
-    if (const char* pp = std::getenv("TT_PINGPONG")) P->pingpong = std::atoi(pp) != 0;
     if (P->variant == 3 && (!tt::attn_2sm_supported(d.head_dim, g) || P->key_tile != 128)) P->variant = 0;
     P->C = d.num_ctas > 0 ? d.num_ctas : P->sm_count;
     if (P->variant == 3) {

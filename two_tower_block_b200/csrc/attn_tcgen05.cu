@@ -15,8 +15,9 @@
 //                key tile into a ring of shared-memory slots (128-byte swizzle);
 //                for a tile whose valid rows are not a multiple of 16 it zeroes
 //                the V rows the last MMA k-step would otherwise read.
-//   warp 1       TMEM owner and MMA issuer (one thread): S = Q_m K^T into TMEM,
-//                O_m += P V with P read from TMEM (aliasing its S buffer).
+//   warp 1       TMEM owner; lane 0 issues the MMAs of M-tile 0: S = Q_0 K^T into
+//                TMEM, O_0 += P V with P read from TMEM (aliasing its S buffer)
+//   warp 2       lane 0 issues the MMAs of M-tile 1 (when the unit has two)
 //   warps 4..7   softmax warpgroup of M-tile 0 (thread = TMEM lane = row)
 //   warps 8..11  softmax warpgroup of M-tile 1
 // TMEM columns: M-tile m owns S buffers [128m, 128m+128) (NBUF buffers of NK
@@ -27,13 +28,6 @@
 // buffer PV(j) has just consumed; with two buffers the softmax of tile j+1
 // finds its S ready while the tensor core works on PV(j).
 //
-// Ping-pong: with two M-tiles the softmax warpgroups take turns at the
-// exponentials (tile G of warpgroup 1 after tile G of warpgroup 0, tile G+1 of
-// warpgroup 0 after that).  Without it both warpgroups receive their scores at
-// the same moment, share the MUFU for the whole tile and leave the tensor core
-// idle meanwhile; with it one M-tile's PV and next S run on the tensor core
-// while the other M-tile's softmax runs.
-//
 // The softmax keeps a running reference maximum per row and rescales O (in
 // TMEM) only when a new maximum exceeds it by more than 2^8; the final
 // normalisation divides by the sum of the same bf16-rounded weights the PV
@@ -41,6 +35,8 @@
 //
 // Every wait is bounded (ptx.cuh: mbar_wait); on a timeout the CTA raises the
 // error word, drains what it issued, frees TMEM and returns.
+#include <type_traits>
+
 #include "combine_row.cuh"
 #include "problem.h"
 #include "ptx.cuh"
@@ -79,7 +75,6 @@ struct Bars {
   uint64_t q_full, q_empty, tail, drain;
   uint64_t s_full[2][2], p_full[2][2];  // [M-tile][S buffer]
   uint64_t pv_done[2], o_full[2], o_empty[2];
-  uint64_t turn[2];                     // ping-pong: warpgroup m may start its exponentials
   uint64_t kv_full[16], kv_empty[16];
 };
 
@@ -177,9 +172,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (tid == 0) {
     mbar_init(smem_u32(&bars->q_full), 1);
-    mbar_init(smem_u32(&bars->q_empty), 1);
+    mbar_init(smem_u32(&bars->q_empty), MT);  // one commit per M-tile issuer
     mbar_init(smem_u32(&bars->tail), 1);
-    mbar_init(smem_u32(&bars->drain), 1);
+    mbar_init(smem_u32(&bars->drain), MT);
     for (int m = 0; m < 2; ++m) {
       for (int b = 0; b < 2; ++b) {
         mbar_init(smem_u32(&bars->s_full[m][b]), 1);
@@ -188,11 +183,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(smem_u32(&bars->pv_done[m]), 1);
       mbar_init(smem_u32(&bars->o_full[m]), 1);
       mbar_init(smem_u32(&bars->o_empty[m]), 128);
-      mbar_init(smem_u32(&bars->turn[m]), 4);  // one arrival per warp of the other warpgroup
     }
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(smem_u32(&bars->kv_full[s]), 1);
-      mbar_init(smem_u32(&bars->kv_empty[s]), 1);
+      mbar_init(smem_u32(&bars->kv_empty[s]), MT);
     }
     sh->abort_flag = 0;
     fence_barrier_init();
@@ -312,27 +306,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait(smem_u32(&bars->kv_full[j % C::kStages]), (j / C::kStages) & 1, dw);
       if (q_it) mbar_wait(smem_u32(&bars->q_full), (q_it - 1) & 1, dw);
     }
-  } else if (warp == 1 && have_work) {
-    // ============================================================= MMA warp ==
+  } else if ((warp == 1 || (warp == 2 && MT == 2)) && have_work) {
+    // ====================================================== MMA issuers ==
+    // One thread per M-tile (warp 1 lane 0: M-tile 0, warp 2 lane 0: M-tile 1), so an M-tile
+    // whose P is not ready never holds back the other's MMAs; the tensor core interleaves the
+    // two instruction streams.  Each thread commits its own reads of a ring slot and of Q,
+    // and those barriers expect one commit per M-tile.
     if (lane == 0) {
+      const int m = warp - 1;
       uint32_t it = 0, q_it = 0, G = 0, seg_cnt = 0;
       bool ok = true;
       Unit x = sh->first;
       // descriptors: a start-address offset is added in 16-byte units to the low field
-      const uint64_t qdesc = smem_desc_sw128(q_s, 16, 1024);
+      const uint64_t qdesc = smem_desc_sw128(q_s + m * 128 * kRowBytes, 16, 1024);
       const uint64_t kdesc0 = smem_desc_sw128(kv_s, 16, 1024);
       const uint64_t vdesc0 = smem_desc_sw128(kv_s, NK * kRowBytes, 1024);
       const uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
       const uint32_t idesc_s0 = idesc_bf16_f32(128, 0, 0, 0);
-      auto issue_s = [&](int m, int buf, uint32_t slot, int n_mma) {
+      const uint32_t s_tmem = tmem + m * 128, o_tmem = tmem + 256 + m * D;
+      auto issue_s = [&](int buf, uint32_t slot, int n_mma) {
         const uint32_t idesc = idesc_s0 | ((uint32_t)(n_mma >> 3) << 17);
         const uint64_t kd = kdesc0 + (uint64_t)((slot * C::kSlotBytes) >> 4);
-        const uint64_t qd = qdesc + (uint64_t)((m * 128 * kRowBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * (kMaxRows * kRowBytes) + (kk & 3) * 32;
           const uint32_t koff = (kk >> 2) * (NK * kRowBytes) + (kk & 3) * 32;
-          tc_mma_ss(tmem + m * 128 + buf * NK, qd + (off >> 4), kd + (koff >> 4), idesc, kk > 0);
+          tc_mma_ss(s_tmem + buf * NK, qdesc + (off >> 4), kd + (koff >> 4), idesc, kk > 0);
         }
       };
       auto kv_wait = [&](uint32_t e) {
@@ -352,49 +351,47 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const int nk = round16(tile_keys(p, x, sg.lo + j).count);
           const uint32_t ks = (it + 2 * j) % C::kStages;
-          for (int m = 0; m < MT; ++m) {
-            issue_s(m, (G + j) % NBUF, ks, nk);
-            tc_commit(smem_u32(&bars->s_full[m][(G + j) % NBUF]));
-          }
+          issue_s((G + j) % NBUF, ks, nk);
+          tc_commit(smem_u32(&bars->s_full[m][(G + j) % NBUF]));
           tc_commit(smem_u32(&bars->kv_empty[ks]));
         }
         for (int j = 0; j < n && ok; ++j, ++G) {
           const int b = G % NBUF;
           const uint32_t ev = it + 2 * j + 1;  // V of tile j
           ok = kv_wait(ev);
+          if (ok) ok = mbar_wait(smem_u32(&bars->p_full[m][b]), (G / NBUF) & 1, wc);
+          if (ok && j == 0) ok = mbar_wait(smem_u32(&bars->o_empty[m]), (seg_cnt & 1) ^ 1, wc);
           if (!ok) break;
+          tc_fence_after();
           const int nv = round16(tile_keys(p, x, sg.lo + j).count);
-          const bool ahead = j + NBUF < n;     // S of tile j + NBUF goes into buffer b
-          const uint32_t ek = it + 2 * (j + NBUF);
-          const int nk = ahead ? round16(tile_keys(p, x, sg.lo + j + NBUF).count) : 0;
           const uint64_t vd = vdesc0 + (uint64_t)(((ev % C::kStages) * C::kSlotBytes) >> 4);
-          for (int m = 0; m < MT && ok; ++m) {
-            ok = mbar_wait(smem_u32(&bars->p_full[m][b]), (G / NBUF) & 1, wc);
-            if (ok && j == 0) ok = mbar_wait(smem_u32(&bars->o_empty[m]), (seg_cnt & 1) ^ 1, wc);
+          const uint32_t pa = s_tmem + b * NK;
+          if (nv == NK) {
+#pragma unroll
+            for (int kk = 0; kk < NK / 16; ++kk)
+              tc_mma_ts(o_tmem, pa + kk * 8, vd + (uint64_t)(kk * 16 * kRowBytes >> 4), idesc_pv,
+                        (j > 0 || kk > 0) ? 1u : 0u);
+          } else {
+            for (int kk = 0; kk < nv / 16; ++kk)
+              tc_mma_ts(o_tmem, pa + kk * 8, vd + (uint64_t)(kk * 16 * kRowBytes >> 4), idesc_pv,
+                        (j > 0 || kk > 0) ? 1u : 0u);
+          }
+          tc_commit(smem_u32(&bars->pv_done[m]));
+          tc_commit(smem_u32(&bars->kv_empty[ev % C::kStages]));
+          if (j + NBUF < n) {
+            // S of tile j + NBUF into buffer b, after P V(j) has read P(j) from it (in issue order)
+            const uint32_t ek = it + 2 * (j + NBUF);
+            ok = kv_wait(ek);
             if (!ok) break;
             tc_fence_after();
-            const uint32_t pa = tmem + m * 128 + b * NK;
-            for (int kk = 0; kk < nv / 16; ++kk)
-              tc_mma_ts(tmem + 256 + m * D, pa + kk * 8, vd + (uint64_t)(kk * 16 * kRowBytes >> 4), idesc_pv,
-                        (j > 0 || kk > 0) ? 1u : 0u);
-            tc_commit(smem_u32(&bars->pv_done[m]));
-            if (ahead) {
-              if (m == 0) {
-                ok = kv_wait(ek);
-                if (!ok) break;
-                tc_fence_after();
-              }
-              issue_s(m, b, ek % C::kStages, nk);
-              tc_commit(smem_u32(&bars->s_full[m][b]));
-            }
+            issue_s(b, ek % C::kStages, round16(tile_keys(p, x, sg.lo + j + NBUF).count));
+            tc_commit(smem_u32(&bars->s_full[m][b]));
+            tc_commit(smem_u32(&bars->kv_empty[ek % C::kStages]));
           }
-          if (!ok) break;
-          tc_commit(smem_u32(&bars->kv_empty[ev % C::kStages]));
-          if (ahead) tc_commit(smem_u32(&bars->kv_empty[ek % C::kStages]));
         }
         if (!ok) break;
         it += 2 * n;
-        for (int m = 0; m < MT; ++m) tc_commit(smem_u32(&bars->o_full[m]));
+        tc_commit(smem_u32(&bars->o_full[m]));
         tc_commit(smem_u32(&bars->q_empty));
         ++seg_cnt;
         if (sg.last) break;
@@ -415,8 +412,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = q4 * 32 + lane;      // row within the M-tile
     const int r = m * 128 + row;         // packed row of the unit
     if (m < MT) {
-      const bool pp = MT == 2 && p.pingpong != 0;
-      const uint32_t turn_mine = smem_u32(&bars->turn[m]), turn_other = smem_u32(&bars->turn[m ^ 1]);
       const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
       const uint32_t s_base = tmem + lane_off + m * 128;  // + buffer * NK
       const uint32_t o_addr = tmem + lane_off + 256 + m * D;
@@ -427,29 +422,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (; ok;) {
         const Segment sg = segment_of(x, start, end, c);
         float m_ref = -INFINITY, l = 0.f;
-        for (int i = sg.lo; i < sg.hi; ++i, ++G) {
-          const int count = tile_keys(p, x, i).count;
-          const int b = G % NBUF;
-          const uint32_t s_addr = s_base + b * NK;
-          ok = mbar_wait(smem_u32(&bars->s_full[m][b]), (G / NBUF) & 1, wc);
-          if (!ok) break;
-          tc_fence_after();
-          // the tile's S row in registers; row maximum in log2 units (masked beyond `count`)
-          const bool full = count == NK;
+        // One tile of the softmax: its S row in registers, the row maximum in log2 units, the
+        // lazy rescale of O, then P (bf16) over the S buffer.  Full tiles and the masked last
+        // tile of a unit run separate code: folding them into one path would make every full
+        // tile pay for the masking.
+        auto tile = [&](auto full_tag, int count, uint32_t s_addr, bool first) -> bool {
+          constexpr bool kFull = decltype(full_tag)::value;
           uint32_t v[NK];
 #pragma unroll
           for (int ch = 0; ch < NK / 32; ++ch)
-            if (full || 32 * ch < count) tmem_ld32(s_addr + 32 * ch, v + 32 * ch);
+            if (kFull || 32 * ch < count) tmem_ld32(s_addr + 32 * ch, v + 32 * ch);
           tc_wait_ld();
-          const float mx = (full ? tile_row_max<NK, true>(v, count) : tile_row_max<NK, false>(v, count)) * p.scale_log2;
-          if (i == sg.lo) {
+          const float mx = tile_row_max<NK, kFull>(v, count) * p.scale_log2;
+          if (first) {
             m_ref = mx;  // O is overwritten by the first PV of the segment
           } else {
             const bool need = mx > m_ref + kRescaleThreshold;
             if (__any_sync(0xffffffffu, need)) {
               // O must hold every earlier PV of this segment before it is rescaled
-              ok = mbar_wait(smem_u32(&bars->pv_done[m]), (G - 1) & 1, wc);
-              if (!ok) break;
+              if (!mbar_wait(smem_u32(&bars->pv_done[m]), (G - 1) & 1, wc)) return false;
               tc_fence_after();
               const float alpha = need ? fast_exp2(m_ref - mx) : 1.f;
               if (need) {
@@ -467,19 +458,24 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
             }
           }
-          // ping-pong turn: warpgroup 0 runs the exponentials of its tile G once warpgroup 1
-          // finished those of tile G-1 (completion G-1 of turn[0]); warpgroup 1 those of tile G
-          // once warpgroup 0 finished tile G (completion G of turn[1]).  Warpgroup 0 starts.
-          if (pp && (m == 1 || G > 0)) {
-            ok = mbar_wait(turn_mine, (m == 0 ? G - 1 : G) & 1, wc);
-            if (!ok) break;
-          }
-          l += full ? tile_exp_store<NK, true>(v, count, p.scale_log2, m_ref, s_addr)
-                    : tile_exp_store<NK, false>(v, count, p.scale_log2, m_ref, s_addr);
-          if (pp) {
-            __syncwarp();
-            if (lane == 0) mbar_arrive(turn_other);
-          }
+          l += tile_exp_store<NK, kFull>(v, count, p.scale_log2, m_ref, s_addr);
+          return true;
+        };
+        for (int i = sg.lo; i < sg.hi; ++i, ++G) {
+          const int count = tile_keys(p, x, i).count;
+          const int b = G % NBUF;
+          const uint32_t s_addr = s_base + b * NK;
+          ok = mbar_wait(smem_u32(&bars->s_full[m][b]), (G / NBUF) & 1, wc);
+          if (!ok) break;
+          tc_fence_after();
+          // (128-key tiles keep a single masked path: a second copy of their 128-register body
+          // would not fit the register budget)
+          if constexpr (NK == 128)
+            ok = tile(std::false_type{}, count, s_addr, i == sg.lo);
+          else
+            ok = count == NK ? tile(std::true_type{}, count, s_addr, i == sg.lo)
+                             : tile(std::false_type{}, count, s_addr, i == sg.lo);
+          if (!ok) break;
           tc_wait_st();
           tc_fence_before();
           mbar_arrive(smem_u32(&bars->p_full[m][b]));

@@ -12,9 +12,11 @@ namespace tt {
 enum Mode : int { kDecode = 0, kBlockCausal = 1 };
 
 // Keys per pipeline tile of each kernel (the work split counts tiles of this size).
-// The tcgen05 kernel also runs with 64-key tiles and two S buffers per M-tile
-// (see tcgen05_key_tile_supported); 128 is the default.
-constexpr int kTcgen05KeyTile = 128;
+// The default tcgen05 kernel runs 64-key tiles with two S buffers per M-tile, so the
+// scores of tile j+1 are computed while the softmax works on tile j; it also runs
+// 128-key tiles with one S buffer (see tcgen05_key_tile_supported), which the
+// transposed-PV and 2-SM forms require.
+constexpr int kTcgen05KeyTile = 64;
 constexpr int kMmaSyncKeyTile = 64;
 
 struct Problem {
@@ -47,8 +49,6 @@ struct Problem {
   unsigned long long wait_limit_ns;
   int variant;          // tcgen05 kernel: 0 = S/P aliasing in TMEM (default), 2 = transposed PV,
                         // 3 = 2-SM pairs (head_dim 128)
-  int pingpong;         // default tcgen05 kernel with two M-tiles: the softmax warpgroups take turns
-                        // at the exponentials, so one M-tile's MMAs run during the other's softmax
   // default tcgen05 kernel launched cooperatively: the CTAs meet at this grid barrier
   // (a counter that only grows) and combine the cut units themselves; null: the
   // separate combine kernel runs instead

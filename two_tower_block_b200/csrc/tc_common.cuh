@@ -19,20 +19,36 @@ __device__ __forceinline__ float* out_row(const Problem& p, const Unit& x, const
   return p.part_o + ((size_t)sg.slot * p.R + r) * D;
 }
 
+// Two non-negative finite weights rounded to bf16 precision on the integer pipe (round half
+// up on the magnitude: add half a bf16 ulp, clear the low 16 bits), returned as fp32 bit
+// patterns whose high halves are the bf16 values.  This keeps the packed conversion off the
+// pipe the exponentials use; only exact ties round differently from round-to-nearest-even.
+__device__ __forceinline__ uint2 round_pair_bf16(float a, float b) {
+  return make_uint2((__float_as_uint(a) + 0x8000u) & 0xFFFF0000u, (__float_as_uint(b) + 0x8000u) & 0xFFFF0000u);
+}
+
 // Row maximum of the first `count` raw scores of a tile (all NK when kFull).
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 template <int NK, bool kFull>
 __device__ __forceinline__ float tile_row_max(const uint32_t* v, int count) {
+  // four running maxima, each taking two new scores per three-input max
   float m[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-  for (int k = 0; k < NK; ++k) {
-    const float x = __uint_as_float(v[k]);
-    m[k & 3] = fmaxf(m[k & 3], (kFull || k < count) ? x : -INFINITY);
+  for (int k = 0; k < NK; k += 2) {
+    const float x0 = (kFull || k < count) ? __uint_as_float(v[k]) : -INFINITY;
+    const float x1 = (kFull || k + 1 < count) ? __uint_as_float(v[k + 1]) : -INFINITY;
+    m[(k >> 1) & 3] = max3f(m[(k >> 1) & 3], x0, x1);
   }
   return fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
 }
 
-// p = 2^(s*c - m_ref) for the tile's keys (0 beyond `count`), rounded to bf16 and
-// written to TMEM as pairs over the first columns of the S buffer: keys
+// p = 2^(s*c - m_ref) for the tile's keys (0 beyond `count`), rounded to bf16
+// (round_pair_bf16) and written to TMEM as pairs over the first columns of the S buffer: keys
 // [32ch, 32ch+32) -> columns [16ch, 16ch+16).  Returns the row sum of the
 // rounded weights, so that numerator and denominator use the same values.
 template <int NK, bool kFull>
@@ -54,9 +70,9 @@ __device__ __forceinline__ float tile_exp_store(const uint32_t* v, int count, fl
         a = c0 < count ? a : 0.f;
         b = c0 + 1 < count ? b : 0.f;
       }
-      const uint32_t h = pack_bf16(a, b);
-      pk[k] = h;
-      acc = __fadd2_rn(acc, make_float2(__uint_as_float(h << 16), __uint_as_float(h & 0xFFFF0000u)));
+      const uint2 r = round_pair_bf16(a, b);
+      pk[k] = __byte_perm(r.x, r.y, 0x7632);
+      acc = __fadd2_rn(acc, make_float2(__uint_as_float(r.x), __uint_as_float(r.y)));
     }
     tmem_st16(s_addr + 16 * ch, pk);
   }
@@ -80,9 +96,9 @@ __device__ __forceinline__ float tile_exp_pack(const uint32_t* v, int count, flo
       a = c0 < count ? a : 0.f;
       b = c0 + 1 < count ? b : 0.f;
     }
-    const uint32_t h = pack_bf16(a, b);
-    pk[k] = h;
-    acc = __fadd2_rn(acc, make_float2(__uint_as_float(h << 16), __uint_as_float(h & 0xFFFF0000u)));
+    const uint2 r = round_pair_bf16(a, b);
+    pk[k] = __byte_perm(r.x, r.y, 0x7632);
+    acc = __fadd2_rn(acc, make_float2(__uint_as_float(r.x), __uint_as_float(r.y)));
   }
   return acc.x + acc.y;
 }
