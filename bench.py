@@ -365,12 +365,12 @@ class Measured:
         n_c, ms_c = self.plan.profile_read(1) if self.info.num_ctas > 1 else (0, 0.0)
         self.plan.profile(False)
         self.plan.check()
+        self.graphs_used = graphs is not None
         del graphs
         self.ms_step = max_over_ranks(pg, ms_total, dev) / args.steps
         self.k_ms = ms_k / max(n_k, 1)
         self.c_ms = ms_c / max(n_c, 1) if n_c else None
         self.launches_per_step = (n_k + n_c) // max(args.steps, 1)
-        self.graphs_used = graphs is not None or not args.no_graph
 
     def record(self, world, peaks):
         value = replica_rate(world, self.cost["bytes"], self.ms_step) / 1e9

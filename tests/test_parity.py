@@ -329,26 +329,42 @@ def test_kv_append_then_decode_equals_decode_with_block_in_context():
 
 
 # --- block-causal backward ------------------------------------------------------------
-def run_backward(inp, dout_bits, kernel=(ops.KERNEL_TCGEN05, {})):
+def run_backward(inp, dout_bits, kernel=(ops.KERNEL_TCGEN05, {}), bwd="tcgen05"):
+    """Forward and backward through the C ABI.  bwd: "tcgen05" (the tensor-memory kernel,
+    where the shape allows it) or "mma_sync" (the warp-level kernel, TT_BWD_KERNEL)."""
     B, N, Hq, D = inp.q.shape
     Hkv = inp.k_ctx.shape[1]
     plan = make_plan(kernel, B, Hq, Hkv, D, inp.block_size, seq_len=N)
     q, kc, vc, kb, vb = dev(inp.q), dev(inp.k_ctx), dev(inp.v_ctx), dev(inp.k_blk), dev(inp.v_blk)
     out, lse = plan.block_attn_block_causal(q, kc, vc, kb, vb, want_lse=True)
-    dq, dk, dv = plan.block_causal_backward(q, kc, vc, kb, vb, out, lse, dev(dout_bits))
-    plan.check()
+    old = os.environ.pop("TT_BWD_KERNEL", None)
+    try:
+        if bwd == "mma_sync":
+            os.environ["TT_BWD_KERNEL"] = "mma_sync"
+        dq, dk, dv = plan.block_causal_backward(q, kc, vc, kb, vb, out, lse, dev(dout_bits))
+        plan.check()
+    finally:
+        os.environ.pop("TT_BWD_KERNEL", None)
+        if old is not None:
+            os.environ["TT_BWD_KERNEL"] = old
     return dq, dk, dv
 
 
+@pytest.mark.parametrize("bwd", ["tcgen05", "mma_sync"])
 @pytest.mark.parametrize("shape", [(2, 64, 16, 8, 2, 128), (1, 40, 4, 8, 1, 64), (2, 300, 20, 4, 2, 128),
-                                   (1, 256, 128, 2, 1, 64)],
-                         ids=["S16-g4-D128", "S4-g8-D64", "S20-g2-D128-ragged", "S128-g2-D64"])
-def test_block_causal_backward_small(shape):
+                                   (1, 256, 128, 2, 1, 64), (1, 128, 16, 16, 1, 128), (2, 96, 16, 32, 2, 64),
+                                   (1, 200, 8, 24, 1, 128)],
+                         ids=["S16-g4-D128", "S4-g8-D64", "S20-g2-D128-ragged", "S128-g2-D64",
+                              "S16-g16-D128-two-Mtiles", "S16-g16-D64-two-Mtiles", "S8-g24-D128-partial-Mtile"])
+def test_block_causal_backward_small(shape, bwd):
+    """Small shapes spanning several key tiles, ragged tails (S = 20: blocks and context tiles
+    that are not multiples of 16), both head dims, one and two 128-row M-tiles (S*g = 256) and
+    a partial second M-tile (S*g = 192, g = 24 does not divide 128: the warp-level kernel)."""
     from oracle import block_causal_backward
     B, N, S, Hq, Hkv, D = shape
     inp = make_causal(B, N, S, Hq, Hkv, D, seed=41)
     dout = bf16_bits(np.random.default_rng(42).standard_normal((B, N, Hq, D)).astype(np.float32))
-    dq, dk, dv = run_backward(inp, dout)
+    dq, dk, dv = run_backward(inp, dout, bwd=bwd)
     rq, rk, rv = block_causal_backward(f64(inp.q), f64(inp.k_ctx), f64(inp.v_ctx), f64(inp.k_blk),
                                        f64(inp.v_blk), f64(dout), S)
     errs = {w: errors(a, r) for w, a, r in (("dq", dq, rq), ("dk_blk", dk, rk), ("dv_blk", dv, rv))}

@@ -592,8 +592,33 @@ tt_status_t tt_block_attn_block_causal_backward(tt_plan_t plan, const void* q, c
   cudaError_t e = cudaMemsetAsync(dk_blk, 0, kv_bytes, s);
   if (e == cudaSuccess) e = cudaMemsetAsync(dv_blk, 0, kv_bytes, s);
   if (e != cudaSuccess) return cuda_fail(e, "clearing dk_blk / dv_blk");
+  p.err_word = plan->err_word;
+  p.wait_limit_ns = (unsigned long long)(d.wait_timeout_us > 0 ? d.wait_timeout_us : 1000000) * 1000ull;
+  // tcgen05 backward on sm_100 plans whose shape it covers (TT_BWD_KERNEL=mma_sync selects
+  // the warp-level kernel); the warp-level kernel takes every other shape
+  bool use_tc = plan->kernel == TT_KERNEL_TCGEN05 && tt::attn_bwd_tc_supported(p);
+  if (const char* bk = std::getenv("TT_BWD_KERNEL")) use_tc = use_tc && std::strcmp(bk, "mma_sync") != 0;
+  tt::BwdMaps maps;
+  if (use_tc) {
+    memset(&maps, 0, sizeof(maps));
+    const uint64_t D = p.D;
+    const uint32_t tpm = p.R > 128 ? 128u / (uint32_t)p.g : (uint32_t)p.S;   // tokens of one M-tile
+    uint64_t qd[3] = {D, (uint64_t)p.Hq, (uint64_t)p.B * p.N};
+    uint64_t qs[2] = {D * 2, (uint64_t)p.Hq * D * 2};
+    uint32_t qb[3] = {64, (uint32_t)p.g, tpm};
+    uint64_t cd[2] = {D, (uint64_t)p.B * p.Hkv * p.N};
+    uint64_t cs[1] = {D * 2};
+    uint32_t cb[2] = {64, 64};
+    uint64_t bd[3] = {D, (uint64_t)p.Hkv, (uint64_t)p.B * p.N};
+    uint64_t bs[2] = {D * 2, (uint64_t)p.Hkv * D * 2};
+    uint32_t bb[3] = {64, 1, (uint32_t)std::min(p.S, 64)};
+    if (!encode_bf16(&maps.q, p.q, 3, qd, qs, qb) || !encode_bf16(&maps.dout, p.dout, 3, qd, qs, qb) ||
+        !encode_bf16(&maps.k_ctx, p.k_ctx, 2, cd, cs, cb) || !encode_bf16(&maps.v_ctx, p.v_ctx, 2, cd, cs, cb) ||
+        !encode_bf16(&maps.k_blk, p.k_blk, 3, bd, bs, bb) || !encode_bf16(&maps.v_blk, p.v_blk, 3, bd, bs, bb))
+      return fail(TT_ERR_CUDA, "tensor map (backward) encode failed");
+  }
   prof_mark(plan, 2, s, true);
-  e = tt::launch_attn_bwd(p, s);
+  e = use_tc ? tt::launch_attn_bwd_tc(p, maps, plan->sm_count, s) : tt::launch_attn_bwd(p, s);
   prof_mark(plan, 2, s, false);
   if (e != cudaSuccess) return cuda_fail(e, "backward kernel launch");
   return TT_OK;
