@@ -15,7 +15,8 @@
 //                (tile 0 = the block's own keys, tiles 1.. = its visible context, 64
 //                keys each) into a ring of shared-memory slots (128-byte swizzle)
 //   warp 1       TMEM owner and MMA issuer (one thread):
-//                  S(j) = Q K(j)^T and dP(j) = dO V(j)^T into TMEM buffer j % 2,
+//                  S(j) = Q K(j)^T and dP(j) = dO V(j)^T into TMEM buffer j % 2 with Q
+//                  and dO read from TMEM (A operands), K and V from shared memory,
 //                  dQ += dS(j) K(j) with dS read from TMEM as a bf16 pair hi + lo
 //   warps 2, 3   block reducer: dK = scale dS^T Q and dV = P^T dO over the item's rows
 //                for the block's own keys (fp32 FMAs on the staged P and dS), added to
@@ -23,11 +24,17 @@
 //                heads of a KV head all contribute)
 //   warps 4..7   softmax warpgroup of the even tiles, warps 8..11 of the odd tiles
 //                (thread = TMEM lane = row): p, ds, dS hi + lo back over the S buffer
-// TMEM columns: S(b) = [64b, 64b+64), dP(b) = [128+64b, ...), dQ = [256, 256+D).
+// TMEM columns: S(b) = [64b, 64b+64), dP(b) = [128+64b, ...) for two buffers b,
+// dQ = [256, 256+D), Q = [384, 384+D/2), dO = [448, 448+D/2) (bf16 pairs).  Q and dO
+// in TMEM leave each S and dP MMA reading only its K or V slice from shared memory.
+// At the start of an item warpgroup 0 copies the item's Q rows and warpgroup 1 its
+// dO rows from the TMA-loaded shared tiles into TMEM.
 //
 // dS enters dQ as hi + lo so dq carries only the rounding of the bf16 inputs; the block
 // reducer takes P and dS in fp32.  Every wait is bounded (ptx.cuh: mbar_wait); on a
 // timeout the CTA raises the error word, drains what it issued, frees TMEM and returns.
+#include <type_traits>
+
 #include "attn_bwd.h"
 
 #include "errbits.h"
@@ -59,7 +66,7 @@ struct BwdCfg {
 };
 
 struct BwdBars {
-  uint64_t q_full, q_empty, dq_full, dq_empty, blk_full, blk_empty, drain;
+  uint64_t q_full, q_empty, qo_full, qo_empty, dq_full, dq_empty, blk_full, blk_empty, drain;
   uint64_t sd_full[2], ds_full[2];
   uint64_t kv_full[kStages], kv_empty[kStages];
 };
@@ -105,12 +112,6 @@ __device__ __forceinline__ void tile_range(const BwdProblem& p, const Item& it, 
 
 __device__ __forceinline__ int round16(int x) { return (x + 15) & ~15; }
 
-// Two fp32 values as a bf16 pair (low half = x0) and the bf16 pair of their remainders.
-__device__ __forceinline__ void split_hi_lo(float x0, float x1, uint32_t& hi, uint32_t& lo) {
-  hi = pack_bf16(x0, x1);
-  lo = pack_bf16(x0 - __uint_as_float(hi << 16), x1 - __uint_as_float(hi & 0xFFFF0000u));
-}
-
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_bwd_tc_kernel(const BwdProblem p, const __grid_constant__ BwdMaps maps) {
@@ -134,7 +135,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   fence_proxy_async_smem();
   if (tid == 0) {
     mbar_init(smem_u32(&bars->q_full), 1);
-    mbar_init(smem_u32(&bars->q_empty), 65);    // MMA commit + the 64 reducer threads
+    mbar_init(smem_u32(&bars->q_empty), 64 + 256);   // the reducer and the two TMEM copies read it
+    mbar_init(smem_u32(&bars->qo_full), 256);         // Q and dO rows written to TMEM
+    mbar_init(smem_u32(&bars->qo_empty), 1);          // the item's last S and dP have read them
     mbar_init(smem_u32(&bars->dq_full), 1);
     mbar_init(smem_u32(&bars->dq_empty), 256);  // both softmax warpgroups read their half
     mbar_init(smem_u32(&bars->blk_full), 128);
@@ -244,11 +247,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       uint32_t it_kv = 0, q_it = 0, G = 0, item_cnt = 0;
       bool ok = true;
-      const uint64_t qdesc = smem_desc_sw128(q_s, 16, 1024);
-      const uint64_t odesc = smem_desc_sw128(o_s, 16, 1024);
+      const uint32_t q_tmem = tmem + 384, o_tmem = tmem + 448;
       const uint64_t kdesc0 = smem_desc_sw128(kv_s, 16, 1024);              // K-major (S, dP)
       const uint64_t kmn0 = smem_desc_sw128(kv_s, kNK * kRowBytes, 1024);   // MN-major (dQ)
-      const uint32_t idesc_sd0 = idesc_bf16_f32(128, 0, 0, 0);
+      const uint32_t idesc_sd0 = idesc_bf16_f32(128, 0, 0, 0);   // A (Q, dO) from TMEM, K-major B
       const uint32_t idesc_dq = idesc_bf16_f32(128, D, 0, 1);
       const uint32_t dq_tmem = tmem + 256;
       // S = Q K^T and dP = dO V^T of tile j into buffer b (K, V = ring entries ek, ek + 1)
@@ -258,15 +260,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t vd = kdesc0 + (uint64_t)((((ek + 1) % kStages) * C::kSlotBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * (128 * kRowBytes) + (kk & 3) * 32;
           const uint32_t koff = (kk >> 2) * (kNK * kRowBytes) + (kk & 3) * 32;
-          tc_mma_ss(tmem + 64 * b, qdesc + (off >> 4), kd + (koff >> 4), idesc, kk > 0);
+          tc_mma_ts(tmem + 64 * b, q_tmem + kk * 8, kd + (koff >> 4), idesc, kk > 0);
         }
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * (128 * kRowBytes) + (kk & 3) * 32;
           const uint32_t koff = (kk >> 2) * (kNK * kRowBytes) + (kk & 3) * 32;
-          tc_mma_ss(tmem + 128 + 64 * b, odesc + (off >> 4), vd + (koff >> 4), idesc, kk > 0);
+          tc_mma_ts(tmem + 128 + 64 * b, o_tmem + kk * 8, vd + (koff >> 4), idesc, kk > 0);
         }
       };
       auto kv_wait = [&](uint32_t e) {
@@ -275,7 +275,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x, ++item_cnt) {
         const Item x = item_of(p, idx, MT);
         const int n = x.tiles;
-        ok = mbar_wait(smem_u32(&bars->q_full), q_it & 1, wc);
+        ok = mbar_wait(smem_u32(&bars->qo_full), q_it & 1, wc);
         ++q_it;
         if (!ok) break;
         tc_fence_after();
@@ -326,7 +326,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         it_kv += 2 * n;
         tc_commit(smem_u32(&bars->dq_full));
-        tc_commit(smem_u32(&bars->q_empty));
+        tc_commit(smem_u32(&bars->qo_empty));
       }
       tc_commit(smem_u32(&bars->drain));
       int dummy = 0;
@@ -393,12 +393,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ========================================================= softmax WGs ==
-    const int w = (warp - 4) >> 2;        // this warpgroup takes the CTA's tiles of parity w (TMEM buffer w)
+    const int w = (warp - 4) >> 2;        // this warpgroup takes the CTA's tiles of parity w
     const int q4 = warp & 3;
     const int row = q4 * 32 + lane;       // row within the M-tile = TMEM lane
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
-    const uint32_t s_addr = tmem + lane_off + 64 * w;
-    const uint32_t dp_addr = tmem + lane_off + 128 + 64 * w;
     const uint32_t dq_addr = tmem + lane_off + 256 + (D / 2) * w;
     uint32_t G = 0, item_cnt = 0;
     bool ok = true;
@@ -424,20 +422,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         delta = acc;
       }
-      // item tile j is the CTA's tile G + j and uses buffer (G + j) % 2
-      for (int j = (w ^ (int)(G & 1u)) & 1; j < x.tiles; j += 2) {
-        const uint32_t Gj = G + (uint32_t)j;   // this CTA's global tile index of tile j
-        ok = mbar_wait(smem_u32(&bars->sd_full[w]), (Gj >> 1) & 1, wc);
-        if (!ok) break;
-        tc_fence_after();
-        int first, count;
-        tile_range(p, x, j, first, count);
-        const bool blk = j == 0;
-        if (blk) {
-          // the reducer must be done with the previous item's staged block tile
-          if (item_cnt > 0) ok = mbar_wait(smem_u32(&bars->blk_empty), (item_cnt - 1) & 1, wc);
-          if (!ok) break;
-        }
+      const float2 c2 = make_float2(p.scale_log2, p.scale_log2);
+      const float2 nl2 = make_float2(-lse2, -lse2), nd2 = make_float2(-delta, -delta);
+      // One tile: p = 2^(s c - lse2), ds = p (dp - Delta) for the 64 keys of this row, dS
+      // back to TMEM as hi (columns [0, 32)) and lo ([32, 64)) over the consumed scores.
+      // A full tile runs without masking; in a partial one, keys past `count` take 0 by
+      // selection (their scores and dP come from rows that may hold anything).
+      auto tile = [&](auto full_tag, uint32_t s_addr, uint32_t dp_addr, int count, bool blk) {
+        constexpr bool kFull = decltype(full_tag)::value;
         uint32_t lo0[16];
 #pragma unroll
         for (int ch = 0; ch < 2; ++ch) {
@@ -449,20 +441,23 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int k = 0; k < 16; ++k) {
             const int c0 = 32 * ch + 2 * k;
-            // masked keys and rows take 0 by selection: the scores and dP of keys past `count`
-            // come from rows that may hold anything
-            const bool v0 = valid && c0 < count, v1 = valid && c0 + 1 < count;
-            const float p0 = v0 ? fast_exp2(__uint_as_float(sv[2 * k]) * p.scale_log2 - lse2) : 0.f;
-            const float p1 = v1 ? fast_exp2(__uint_as_float(sv[2 * k + 1]) * p.scale_log2 - lse2) : 0.f;
-            const float d0 = v0 ? p0 * (__uint_as_float(dv[2 * k]) - delta) : 0.f;
-            const float d1 = v1 ? p1 * (__uint_as_float(dv[2 * k + 1]) - delta) : 0.f;
-            split_hi_lo(d0, d1, hi[k], lo[k]);
-            if (blk && c0 < p.S) {
-              stage_p[row * kStageLd + c0] = p0;
-              stage_ds[row * kStageLd + c0] = d0;
+            const float2 xs = __ffma2_rn(make_float2(__uint_as_float(sv[2 * k]), __uint_as_float(sv[2 * k + 1])), c2, nl2);
+            float2 pp = make_float2(fast_exp2(xs.x), fast_exp2(xs.y));
+            float2 dd = __fmul2_rn(pp, __fadd2_rn(make_float2(__uint_as_float(dv[2 * k]), __uint_as_float(dv[2 * k + 1])), nd2));
+            if (!kFull) {
+              const bool v0 = c0 < count, v1 = c0 + 1 < count;
+              pp = make_float2(v0 ? pp.x : 0.f, v1 ? pp.y : 0.f);
+              dd = make_float2(v0 ? dd.x : 0.f, v1 ? dd.y : 0.f);
+            }
+            hi[k] = pack_bf16(dd.x, dd.y);
+            const float2 rem = __fadd2_rn(dd, make_float2(-__uint_as_float(hi[k] << 16), -__uint_as_float(hi[k] & 0xFFFF0000u)));
+            lo[k] = pack_bf16(rem.x, rem.y);
+            if (!kFull && blk && c0 < p.S) {
+              stage_p[row * kStageLd + c0] = valid ? pp.x : 0.f;
+              stage_ds[row * kStageLd + c0] = valid ? dd.x : 0.f;
               if (c0 + 1 < p.S) {
-                stage_p[row * kStageLd + c0 + 1] = p1;
-                stage_ds[row * kStageLd + c0 + 1] = d1;
+                stage_p[row * kStageLd + c0 + 1] = valid ? pp.y : 0.f;
+                stage_ds[row * kStageLd + c0 + 1] = valid ? dd.y : 0.f;
               }
             }
           }
@@ -477,9 +472,59 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_st16(s_addr + 48, lo);
           }
         }
+      };
+      // ---- this item's Q (warpgroup 0) or dO (warpgroup 1) rows into TMEM ----
+      ok = mbar_wait(smem_u32(&bars->q_full), item_cnt & 1, wc);
+      if (ok && item_cnt > 0) ok = mbar_wait(smem_u32(&bars->qo_empty), (item_cnt - 1) & 1, wc);
+      if (!ok) break;
+      tc_fence_after();
+      {
+        const uint8_t* src = smem + (w == 0 ? C::kQOff : C::kOOff);
+        const uint32_t dst = tmem + lane_off + (w == 0 ? 384 : 448);
+#pragma unroll
+        for (int hf = 0; hf < C::kHalves; ++hf) {
+          uint32_t v[32];
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            // chunk c (dims 8c..8c+7 of this half) of row `row` of a 128-byte-swizzled tile
+            const uint4 u = *reinterpret_cast<const uint4*>(src + hf * (128 * kRowBytes) + row * kRowBytes +
+                                                            ((c ^ (row & 7)) << 4));
+            v[4 * c] = u.x;
+            v[4 * c + 1] = u.y;
+            v[4 * c + 2] = u.z;
+            v[4 * c + 3] = u.w;
+          }
+          tmem_st32(dst + 32 * hf, v);
+        }
         tc_wait_st();
         tc_fence_before();
-        mbar_arrive(smem_u32(&bars->ds_full[w]));
+        mbar_arrive(smem_u32(&bars->qo_full));
+        mbar_arrive(smem_u32(&bars->q_empty));   // this warpgroup is done with the shared tile
+      }
+      // item tile j is the CTA's tile G + j, in TMEM buffer (G + j) % 2
+      for (int j = (w ^ (int)(G & 1u)) & 1; j < x.tiles; j += 2) {
+        const uint32_t Gj = G + (uint32_t)j;
+        const int b = (int)(Gj & 1u);
+        ok = mbar_wait(smem_u32(&bars->sd_full[b]), (Gj >> 1) & 1u, wc);
+        if (!ok) break;
+        tc_fence_after();
+        int first, count;
+        tile_range(p, x, j, first, count);
+        const bool blk = j == 0;
+        if (blk && item_cnt > 0) {
+          // the reducer must be done with the previous item's staged block tile
+          ok = mbar_wait(smem_u32(&bars->blk_empty), (item_cnt - 1) & 1, wc);
+          if (!ok) break;
+        }
+        const uint32_t s_addr = tmem + lane_off + 64 * b, dp_addr = tmem + lane_off + 128 + 64 * b;
+        // the block tile (<= 32 keys) always takes the masked path, which also stages P and dS
+        if (count == kNK && !blk)
+          tile(std::true_type{}, s_addr, dp_addr, count, false);
+        else
+          tile(std::false_type{}, s_addr, dp_addr, count, blk);
+        tc_wait_st();
+        tc_fence_before();
+        mbar_arrive(smem_u32(&bars->ds_full[b]));
         if (blk) {
           __threadfence_block();
           mbar_arrive(smem_u32(&bars->blk_full));
