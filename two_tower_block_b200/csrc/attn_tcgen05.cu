@@ -245,10 +245,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       // paged cache: a context tile is loaded in slices of psub rows, one per page (pages of
       // at least NK keys hold whole tiles); slices past the tile's last key are not loaded
       const int psub = p.page_table ? min(1 << p.page_shift, NK) : NK;
+      // paged context: lane s looks up the pool row of slice s of a tile (one table read per
+      // lane, all in flight together), one tile ahead of the loads that use it
+      auto slice_row = [&](int i) -> int {
+        const TileKeys tk = tile_keys(p, x, i);
+        if (!p.page_table || tk.is_blk || lane * psub >= tk.count) return 0;
+        const int row = paged_row(p, x.n, x.h, tk.first + lane * psub);
+        return row < 0 ? (p.num_pages * p.Hkv) << p.page_shift : row;  // a bad page reads as zeros
+      };
+      int cur_row = slice_row(sg.lo);
       for (int i = sg.lo; i < sg.hi && ok; ++i) {
         const TileKeys tk = tile_keys(p, x, i);
         const int box_rows = tk.is_blk ? min(p.S, NK) : (p.page_table ? ceil_div(tk.count, psub) * psub : NK);
         const uint32_t bytes = (uint32_t)(box_rows * kRowBytes * C::kHalves);
+        const int nsl = p.page_table && !tk.is_blk ? box_rows / psub : 0;   // slices of a paged tile
+        const int row_i = cur_row;
+        if (i + 1 < sg.hi) cur_row = slice_row(i + 1);
         for (int kv = 0; kv < 2 && ok; ++kv, ++it) {
           const int s = it % C::kStages;
           ok = mbar_wait(smem_u32(&bars->kv_empty[s]), ((it / C::kStages) & 1) ^ 1, wc);
@@ -258,21 +270,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           // V rows [count, round16(count)) are read by the last PV k-step: zero them.
           const bool fix = kv == 1 && (tk.count & 15) != 0;
           const uint32_t bar = fix ? smem_u32(&bars->tail) : smem_u32(&bars->kv_full[s]);
-          if (lane == 0) {
-            mbar_arrive_expect_tx(bar, bytes);
+          if (lane == 0) mbar_arrive_expect_tx(bar, bytes);
+          if (nsl > 0) {
+            // each slice lands at its row offset in the stage (a multiple of 2 KB: the swizzle
+            // pattern stays aligned); issued after the expected byte count is set
+            __syncwarp();
+            if (lane < nsl)
+              for (int hf = 0; hf < C::kHalves; ++hf)
+                tma_load_2d(slot + hf * (NK * kRowBytes) + lane * psub * kRowBytes, m, bar, hf * 64, row_i);
+          } else if (lane == 0) {
             for (int hf = 0; hf < C::kHalves; ++hf) {
               const uint32_t dst = slot + hf * (NK * kRowBytes);
-              if (tk.is_blk) {
-                tma_load_3d(dst, m, bar, hf * 64, x.h, x.ns * p.S + tk.first);
-              } else if (!p.page_table) {
-                tma_load_2d(dst, m, bar, hf * 64, ctx_row0 + tk.first);
-              } else {
-                // a page outside the pool reads as zeros (row coordinate past the pool's end)
-                for (int r = 0; r < box_rows; r += psub) {
-                  const int row = paged_row(p, x.n, x.h, tk.first + r);
-                  tma_load_2d(dst + r * kRowBytes, m, bar, hf * 64, row < 0 ? (p.num_pages * p.Hkv) << p.page_shift : row);
-                }
-              }
+              if (tk.is_blk) tma_load_3d(dst, m, bar, hf * 64, x.h, x.ns * p.S + tk.first);
+              else tma_load_2d(dst, m, bar, hf * 64, ctx_row0 + tk.first);
             }
           }
           if (fix) {
