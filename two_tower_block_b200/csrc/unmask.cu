@@ -11,7 +11,10 @@
 // Kernel 1: one CTA per (sequence, position) row that is still masked.  It streams
 // the row's V bf16 logits once with 16-byte loads, keeping an online (max, sum of
 // 2^(x - max), argmax) per thread in the log2 domain, merged across the CTA; the
-// probability of the argmax token is 1 / sum.  Kernel 2: one CTA per sequence
+// probability of the argmax token is 1 / sum.  Each thread takes its logits in batches
+// of 32 (four 16-byte loads in flight), rescaling its sum once per batch; 1024 threads
+// per row keep 64 KB of loads in flight per SM.  Kernel 2 is launched as a
+// programmatic dependent of kernel 1, so its launch overlaps the scan.  Kernel 2: one CTA per sequence
 // applies the commit rule to tokens and mask.
 #include "unmask.h"
 
@@ -22,7 +25,7 @@
 namespace tt {
 namespace {
 
-constexpr int kScanThreads = 512;
+constexpr int kScanThreads = 1024;   // one CTA per row
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct Acc {
@@ -52,9 +55,11 @@ __device__ __forceinline__ Acc acc_merge(const Acc& a, const Acc& b) {
   return r;
 }
 
-__global__ void __launch_bounds__(kScanThreads)
+__global__ void __launch_bounds__(kScanThreads, 1)
     unmask_scan_kernel(const __nv_bfloat16* __restrict__ logits, const uint8_t* __restrict__ masked, int V,
                        float* __restrict__ p_max, int32_t* __restrict__ argmax) {
+  // the commit kernel may be scheduled now; it waits for this grid's results itself
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int row = blockIdx.x;
   if (!masked[row]) {
     if (threadIdx.x == 0) {
@@ -66,28 +71,71 @@ __global__ void __launch_bounds__(kScanThreads)
   const __nv_bfloat16* x = logits + (size_t)row * V;
   Acc a{-INFINITY, 0.f, 0};
   if ((V & 7) == 0) {
+    // batches of kBatch 16-byte loads per thread, all in flight together; per batch one
+    // maximum (and the first index reaching it, in ascending index order), one rescale of
+    // the running sum, then the batch's exponentials as independent pairs
     const uint4* x8 = reinterpret_cast<const uint4*>(x);
-    const int n8 = V >> 3;
-    constexpr int kDepth = 4;   // 16-byte loads a thread has in flight
-    for (int i0 = threadIdx.x; i0 < n8; i0 += kDepth * kScanThreads) {
-      uint4 v[kDepth];
+    const int n8 = V >> 3, lo8 = 0;
+    constexpr int kBatch = 4;
+    const float2 c2 = make_float2(kLog2e, kLog2e);
+    constexpr uint32_t kNegInf2 = 0xFF80FF80u;   // two bf16 -inf
+    for (int base = lo8; base < n8; base += kBatch * kScanThreads) {
+      uint4 v[kBatch];
 #pragma unroll
-      for (int u = 0; u < kDepth; ++u) {
-        const int i = i0 + u * kScanThreads;
-        if (i < n8) v[u] = __ldcs(x8 + i);   // streamed once
+      for (int u = 0; u < kBatch; ++u) {
+        const int i = base + u * kScanThreads + threadIdx.x;
+        v[u] = i < n8 ? __ldcs(x8 + i) : make_uint4(kNegInf2, kNegInf2, kNegInf2, kNegInf2);
       }
+      // batch maximum and the first index reaching it: four independent trackers (one per
+      // 32-bit word of a load), each visiting its values in ascending index order, merged
+      // with the lower index winning ties
+      float bm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      int barg[4] = {0, 0, 0, 0};
 #pragma unroll
-      for (int u = 0; u < kDepth; ++u) {   // ascending index order within the thread
-        const int i = i0 + u * kScanThreads;
-        if (i < n8) {
-          const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+      for (int u = 0; u < kBatch; ++u) {
+        const int i = base + u * kScanThreads + threadIdx.x;
+        const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            acc_push(a, __uint_as_float(w[k] << 16), 8 * i + 2 * k);
-            acc_push(a, __uint_as_float(w[k] & 0xFFFF0000u), 8 * i + 2 * k + 1);
+        for (int k = 0; k < 4; ++k) {
+          const float lo = __uint_as_float(w[k] << 16), hi = __uint_as_float(w[k] & 0xFFFF0000u);
+          if (lo > bm[k]) {
+            bm[k] = lo;
+            barg[k] = 8 * i + 2 * k;
+          }
+          if (hi > bm[k]) {
+            bm[k] = hi;
+            barg[k] = 8 * i + 2 * k + 1;
           }
         }
       }
+#pragma unroll
+      for (int k = 1; k < 4; ++k) {
+        if (bm[k] > bm[0] || (bm[k] == bm[0] && barg[k] < barg[0])) {
+          bm[0] = bm[k];
+          barg[0] = barg[k];
+        }
+      }
+      const float z = bm[0] * kLog2e;
+      if (z > a.m) {
+        a.s *= fast_exp2(a.m - z);
+        a.m = z;
+        a.arg = barg[0];
+      }
+      const float2 nm2 = make_float2(-a.m, -a.m);
+      float2 s0 = make_float2(0.f, 0.f), s1 = s0;
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float2 t = __ffma2_rn(make_float2(__uint_as_float(w[k] << 16), __uint_as_float(w[k] & 0xFFFF0000u)),
+                                      c2, nm2);
+          const float2 e = make_float2(fast_exp2(t.x), fast_exp2(t.y));
+          if (k & 1) s1 = __fadd2_rn(s1, e);
+          else s0 = __fadd2_rn(s0, e);
+        }
+      }
+      a.s += (s0.x + s0.y) + (s1.x + s1.y);
     }
   } else {
     for (int i = threadIdx.x; i < V; i += kScanThreads) acc_push(a, __bfloat162float(x[i]), i);
@@ -121,6 +169,7 @@ __global__ void __launch_bounds__(kScanThreads)
 __global__ void unmask_commit_kernel(int S, float gamma, int min_one, int32_t* tokens, uint8_t* masked,
                                      const float* __restrict__ p_max, const int32_t* __restrict__ argmax,
                                      int32_t* n_committed) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");   // the scan grid's results are complete and visible
   const int n = blockIdx.x, s = threadIdx.x;
   __shared__ unsigned long long best;   // (confidence bits << 32) | (~position): the most confident, first
   __shared__ int any_pass, count;
@@ -157,9 +206,19 @@ cudaError_t launch_confidence_unmask(const void* logits, int B, int S, int V, fl
                                                           p_max, argmax);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const int threads = ((S + 31) / 32) * 32;
-  unmask_commit_kernel<<<B, threads, 0, stream>>>(S, gamma, min_one, tokens, masked, p_max, argmax, n_committed);
-  return cudaGetLastError();
+  // the commit kernel is launched as a programmatic dependent of the scan: its launch
+  // overlaps the scan, and it waits for the scan's results on the device
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(B, 1, 1);
+  cfg.blockDim = dim3(((S + 31) / 32) * 32, 1, 1);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, unmask_commit_kernel, S, gamma, min_one, tokens, masked,
+                            static_cast<const float*>(p_max), static_cast<const int32_t*>(argmax), n_committed);
 }
 
 }  // namespace tt
