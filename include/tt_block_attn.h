@@ -202,8 +202,10 @@ TT_API tt_status_t tt_block_attn_host(tt_plan_t plan, const void* q, const void*
  *   status    optional device uint32: zeroed, then receives the device error
  *             bits (1 = ctx_lens out of range, 2 = a wait timed out); NULL
  *             discards them.
- * Scratch: one file-scope device array of 16 MiB that every GPU loading this
- * library keeps until the process exits.  The first call on a device (with
+ * Scratch: one file-scope device array of 40 MiB that every GPU loading this
+ * library keeps until the process exits (one range per SM of a 148-SM GPU at
+ * S*g = 256 rows and head_dim 128; an automatic split shrinks its range count
+ * to fit).  The first call on a device (with
  * that device current) resolves the array's device address; make that first
  * call before any stream capture.  Every call shares the array and leaves its
  * contents behind, so calls that overlap on the GPU (different streams, or
@@ -291,10 +293,12 @@ TT_API tt_status_t tt_block_attn_profile_read(tt_plan_t plan, int kernel_id, int
  * the device context still usable afterwards. */
 TT_API tt_status_t tt_selftest_wait_timeout(int device, int timeout_us, tt_stream_t stream);
 
-/* Numerics self test: evaluates on the device the FMA-pipe exp2 the softmax uses
- * for a quarter of its weights (range reduction plus a fitted degree-3 polynomial,
- * maximum relative error 7.5e-5 for arguments in [-125, 127]) on the n host values
- * x and writes the n results to y (host).  Synchronous; allocates its own
+/* Numerics self test: evaluates on the device the library's FMA-pipe exp2 (range
+ * reduction plus a fitted degree-3 polynomial, maximum relative error 7.5e-5 for
+ * arguments in [-125, 127]) on the n host values x and writes the n results to y
+ * (host).  The attention kernels do not use it: they call the hardware exp2
+ * (ex2.approx), because offloading part of the softmax's exponentials to the FMA pipe
+ * measured slower.  It stays a tested building block.  Synchronous; allocates its own
  * buffers. */
 TT_API tt_status_t tt_selftest_exp2(int device, const float* x, float* y, int n);
 

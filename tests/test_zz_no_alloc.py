@@ -74,3 +74,47 @@ def test_noalloc_rejects_scratch_beyond_limit():
     st = ops.block_attn_noalloc(*args, out, num_ctas=4096)  # 4096 ranges need ~1 GiB of partials
     assert st == ops.TT_ERR_INVALID_ARG
     assert b"scratch" in ops.lib().tt_last_error_detail()
+
+
+def _oracle(inp):
+    from oracle import block_attn as oracle_attn
+    from tests.gpu_util import f64
+    return oracle_attn(f64(inp.q), f64(inp.k_ctx), f64(inp.v_ctx), f64(inp.k_blk), f64(inp.v_blk), inp.ctx_lens)
+
+
+@pytest.mark.parametrize("kernel", [ops.KERNEL_AUTO, ops.KERNEL_MMA_SYNC], ids=["tcgen05", "mma_sync"])
+@pytest.mark.parametrize("case", ["ragged-gqa16", "no-context", "d64-S5-g3"])
+def test_noalloc_matches_oracle(case, kernel):
+    """Against the float64 oracle directly, at the parity tests' tolerance: ragged GQA rows
+    (context rows past L_n are NaN), a plan shape without any context (ctx_capacity = 0: the
+    context maps stand in for the block's), and head_dim 64 with S = 5, g = 3; both kernels."""
+    inp = {"ragged-gqa16": lambda: make_decode(3, 16, 32, 2, 128, 900, seed=95, ctx_lens=[900, 0, 129]),
+           "no-context": lambda: make_decode(2, 16, 8, 2, 128, 0, seed=96),
+           "d64-S5-g3": lambda: make_decode(2, 5, 6, 2, 64, 300, seed=97, ctx_lens=[300, 17])}[case]()
+    B, S, Hq, Hkv, D, Lcap = inp.shape
+    args = _inputs(inp)
+    out = torch.full((B, S, Hq, D), float("nan"), device="cuda")
+    lse = torch.full((B, Hq, S), float("nan"), device="cuda")
+    status = torch.full((1,), 7, dtype=torch.int32, device="cuda")
+    st = ops.block_attn_noalloc(*args, out, lse, status, kernel=kernel)
+    assert st == ops.TT_OK, ops.lib().tt_last_error_detail()
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    ro, rl = _oracle(inp)
+    assert_parity(out, ro, f"{case} noalloc out vs oracle")
+    assert_parity(lse, rl, f"{case} noalloc lse vs oracle")
+
+
+def test_noalloc_reports_out_of_range_ctx_len():
+    """A ctx_lens value past ctx_capacity reaches the caller's status word (bit 1), and the
+    sequences with valid lengths still match the oracle."""
+    inp = make_decode(2, 16, 16, 1, 128, 256, seed=98, ctx_lens=[256, 100])
+    args = _inputs(inp)
+    bad = torch.tensor([256, 5000], dtype=torch.int32, device="cuda")   # 5000 > ctx_capacity
+    out = torch.empty((2, 16, 16, 128), device="cuda")
+    status = torch.zeros((1,), dtype=torch.int32, device="cuda")
+    assert ops.block_attn_noalloc(*args[:5], bad, out, None, status) == ops.TT_OK
+    torch.cuda.synchronize()
+    assert int(status.item()) & 1
+    ro, _ = _oracle(inp)
+    assert_parity(out[:1], ro[:1], "noalloc out, valid sequence")

@@ -84,6 +84,7 @@ struct tt_plan_s {
   int sm_count = 0;
   int kernel = TT_KERNEL_MMA_SYNC;
   int C = 1;
+  int C_paged = 1;   // ranges of paged calls (differs from C on 2-SM plans)
   int key_tile = 64;
   int variant = 0;
   int R = 0, g = 1;
@@ -218,7 +219,7 @@ tt_status_t launch_all(tt_plan_t plan, const tt::Problem& p, cudaStream_t s) {
   }
   prof_mark(plan, 0, s, false);
   if (e != cudaSuccess) return cuda_fail(e, "attention kernel launch");
-  if (plan->C > 1 && p.grid_bar == nullptr) {
+  if (p.C > 1 && p.grid_bar == nullptr) {
     prof_mark(plan, 1, s, true);
     e = tt::launch_combine(p, s);
     prof_mark(plan, 1, s, false);
@@ -330,11 +331,14 @@ tt_status_t tt_block_attn_plan(const tt_block_attn_desc* desc, int device, tt_pl
     P->causal_T = (long long)d.batch * d.num_kv_heads * acc;
   }
 
-  // scratch layout (256-byte aligned pieces)
+  // scratch layout (256-byte aligned pieces).  A 2-SM plan runs one range per SM pair, but
+  // its paged calls run on the one-CTA-per-SM kernel: room for one range per SM as well.
+  P->C_paged = (P->kernel == TT_KERNEL_TCGEN05 && P->variant == 3 && d.num_ctas <= 0) ? P->sm_count : P->C;
+  const int Cmax = std::max(P->C, P->C_paged);
   auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
-  const size_t b_po = up((size_t)2 * P->C * P->R * d.head_dim * sizeof(float));
-  const size_t b_pl = up((size_t)2 * P->C * P->R * sizeof(float));
-  const size_t b_rec = up((size_t)P->C * sizeof(tt::SplitRecord));
+  const size_t b_po = up((size_t)2 * Cmax * P->R * d.head_dim * sizeof(float));
+  const size_t b_pl = up((size_t)2 * Cmax * P->R * sizeof(float));
+  const size_t b_rec = up((size_t)Cmax * sizeof(tt::SplitRecord));
   const size_t b_err = 256;
   const size_t b_pref = up(pref.size() * sizeof(int));
   P->ws_bytes = b_po + b_pl + b_rec + b_err + b_pref;
@@ -461,6 +465,7 @@ tt_status_t tt_block_attn_paged(tt_plan_t plan, const void* q, const void* k_pag
   p.mode = tt::kDecode;
   p.NB = 1;
   p.variant = 0;  // the paged loads live in the default tcgen05 kernel (and the mma.sync one)
+  p.C = plan->C_paged;
   p.ctx_stride = pages_per_seq * page_size;
   int shift = 0;
   while ((1 << shift) < page_size) ++shift;

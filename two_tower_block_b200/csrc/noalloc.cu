@@ -27,7 +27,8 @@ extern thread_local std::string g_detail;  // shared with the other entry points
 
 namespace {
 
-constexpr size_t kScratchBytes = size_t(16) << 20;  // 16 MiB per device
+// 40 MiB per device: room for one range per SM (148) at S*g = 256 rows and head_dim 128
+constexpr size_t kScratchBytes = size_t(40) << 20;
 constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char g_scratch[kScratchBytes];

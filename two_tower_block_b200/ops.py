@@ -414,7 +414,7 @@ def work_split(tiles_per_unit, num_ctas):
 def block_attn_noalloc(q, k_ctx, v_ctx, k_blk, v_blk, ctx_lens, out, lse=None, status=None, scale=0.0,
                        kernel=KERNEL_AUTO, num_ctas=0, stream=None):
     """Decode through tt_block_attn_noalloc: no plan, no device allocation inside the
-    library (its scratch is a fixed 16 MiB device array).  Outputs are caller-owned;
+    library (its scratch is a fixed 40 MiB device array).  Outputs are caller-owned;
     `status` is an optional one-element uint32/int32 device tensor for the error bits."""
     B, S, Hq, D = q.shape
     Hkv, Lcap = k_ctx.shape[1], k_ctx.shape[2]
