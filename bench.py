@@ -48,6 +48,8 @@ def parse():
     ap.add_argument("--workload", type=int, default=4, choices=[1, 2, 3, 4, 5])
     ap.add_argument("--only", action="store_true", help="time the named workload alone (no per-workload records)")
     ap.add_argument("--no-backward", action="store_true", help="skip the block-causal backward measurement")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="override the workload's batch (same per-sequence recipe): small cases for profiler captures")
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--kernel", default="auto", choices=["auto", "tcgen05", "mma_sync"])
     ap.add_argument("--no-graph", action="store_true", help="launch steps directly instead of via CUDA graphs")
@@ -70,7 +72,8 @@ def load_peaks():
 
 
 def kernel_source_hash(kind: str) -> str:
-    files = {"tcgen05": ["attn_tcgen05.cu"], "tcgen05_pt": ["attn_tcgen05_pt.cu", "tc_common.cuh"],
+    files = {"tcgen05": ["attn_tcgen05.cu", "tc_common.cuh"], "tcgen05_pt": ["attn_tcgen05_pt.cu", "tc_common.cuh"],
+             "bwd_tc": ["attn_bwd_tc.cu", "attn_bwd.h"], "unmask": ["unmask.cu"],
              "tcgen05_2sm": ["attn_tcgen05_2sm.cu", "tc_common.cuh"], "mma_sync": ["attn_mma_sync.cu"]}[kind]
     h = hashlib.sha256()
     for f in files + ["ptx.cuh", "walker.cuh", "problem.h", "sched.cuh"]:
@@ -175,9 +178,10 @@ def replica_rate(world, units_per_replica, ms_max):
 def workload_cost(wid, inp):
     from two_tower_block_b200.workloads import WORKLOADS, causal_cost, decode_cost
     w = WORKLOADS[wid]
+    B = int(inp.q.shape[0])   # the inputs' batch (a --batch override changes it)
     if w.kind == "decode":
-        return decode_cost(w.batch, w.block_size, w.num_q_heads, w.num_kv_heads, w.head_dim, inp.ctx_lens)
-    return causal_cost(w.batch, w.seq_len, w.block_size, w.num_q_heads, w.num_kv_heads, w.head_dim)
+        return decode_cost(B, w.block_size, w.num_q_heads, w.num_kv_heads, w.head_dim, inp.ctx_lens)
+    return causal_cost(B, w.seq_len, w.block_size, w.num_q_heads, w.num_kv_heads, w.head_dim)
 
 
 # --------------------------------------------------------------- oracle arm --
@@ -280,8 +284,11 @@ class Measured:
         from two_tower_block_b200 import ops
         from two_tower_block_b200.workloads import WORKLOADS, make_workload
         self.wid, self.w = wid, WORKLOADS[wid]
+        if args.batch:
+            import dataclasses
+            self.w = dataclasses.replace(self.w, batch=args.batch)
         w = self.w
-        self.inp = make_workload(wid)
+        self.inp = make_workload(wid, batch=args.batch or None)
         self.cost = workload_cost(wid, self.inp)
         self.l2 = torch.cuda.get_device_properties(dev).L2_cache_size
 
