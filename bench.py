@@ -257,21 +257,22 @@ def run_reference(args):
 
 
 # --------------------------------------------------------------- native arm --
-def roofline_of(wid, cost, k_ms, kname, peaks):
+def roofline_of(wid, cost, k_ms, kname, peaks, batch_override=0):
     """Roofline record of the dominant (attention) kernel of one workload: algorithmic bytes
     (decode, HBM-bound) or flops (block-causal, tensor-bound) per launch over its average
     event-timed duration."""
     from two_tower_block_b200.workloads import WORKLOADS
+    traffic = None if batch_override else recorded_traffic(kname, wid)
     if WORKLOADS[wid].kind == "decode":
         achieved = cost["bytes"] / (k_ms * 1e-3) / 1e9
         return {"bound": "hbm", "achieved": round(achieved, 2), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": recorded_traffic(kname, wid),
+                "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": traffic,
                 "kernel": f"attn_{kname}", "kernel_ms": round(k_ms, 5),
                 "peak_source": peaks["source"] + " (hbm_gbs, copy)"}
     ach_t = cost["flops"] / (k_ms * 1e-3) / 1e12
     pk = peaks["bf16_tflops_sustained"] or peaks["bf16_tflops"]
     return {"bound": "tensor", "achieved": round(ach_t, 2), "peak": pk, "unit": "TFLOP/s",
-            "frac": round(ach_t / pk, 4), "traffic": recorded_traffic(kname, wid),
+            "frac": round(ach_t / pk, 4), "traffic": traffic,
             "kernel": f"attn_{kname}", "kernel_ms": round(k_ms, 5),
             "peak_source": peaks["source"] + " (bf16_tflops_sustained, cuBLAS)"}
 
@@ -284,6 +285,7 @@ class Measured:
         from two_tower_block_b200 import ops
         from two_tower_block_b200.workloads import WORKLOADS, make_workload
         self.wid, self.w = wid, WORKLOADS[wid]
+        self.args_batch = args.batch
         if args.batch:
             import dataclasses
             self.w = dataclasses.replace(self.w, batch=args.batch)
@@ -384,7 +386,7 @@ class Measured:
         return {"workload": self.w.name, "value": round(value, 3), "unit": "GB/s",
                 "ms_per_step": round(self.ms_step, 5), "tflops": round(tflops, 2),
                 "alg_bytes": int(self.cost["bytes"]), "flops": int(self.cost["flops"]),
-                "roofline": roofline_of(self.wid, self.cost, self.k_ms, self.kname, peaks),
+                "roofline": roofline_of(self.wid, self.cost, self.k_ms, self.kname, peaks, self.args_batch),
                 "combine_kernel_ms": round(self.c_ms, 5) if self.c_ms else None,
                 "launches_per_step": self.launches_per_step, "num_ctas": self.info.num_ctas,
                 "l2": "inputs rotate over %d copies (%.0f MB) > 2x L2 (%d MB)" % (
@@ -426,8 +428,12 @@ def measure_backward(m, dev):
     pkk = load_peaks()
     pk = pkk["bf16_tflops_sustained"] or pkk["bf16_tflops"]
     del bout, blse, dout, dq, dkb, dvb
-    return {"kernel": "attn_bwd", "ms": round(ms_b, 4), "tflops": round(bflops / (ms_b * 1e-3) / 1e12, 2),
-            "frac_of_sustained_bf16": round(bflops / (ms_b * 1e-3) / 1e12 / pk, 4), "launches": nb_l}
+    # the tcgen05 backward runs on sm_100 plans with S <= 32 unless TT_BWD_KERNEL=mma_sync
+    tc = m.info.kernel == 1 and w.block_size <= 32 and os.environ.get("TT_BWD_KERNEL") != "mma_sync"
+    return {"kernel": "attn_bwd_tc" if tc else "attn_bwd (mma.sync)", "ms": round(ms_b, 4),
+            "tflops": round(bflops / (ms_b * 1e-3) / 1e12, 2),
+            "frac_of_sustained_bf16": round(bflops / (ms_b * 1e-3) / 1e12 / pk, 4), "launches": nb_l,
+            "traffic": recorded_traffic("bwd_tc", m.wid) if tc and not m.args_batch else None}
 
 
 def run_native(args):
@@ -625,6 +631,7 @@ def run_native(args):
         unmask = {"rows": UB * w.block_size, "vocab": Vv, "us_per_call": round(us, 3), "bytes": ubytes,
                   "gbs": round(ubytes / (us * 1e-6) / 1e9, 2),
                   "frac_hbm": round(ubytes / (us * 1e-6) / 1e9 / peaks["hbm_gbs"], 4), "launches_per_call": 2,
+                  "traffic": recorded_traffic("unmask", 0),
                   "l2": "logits rotate over %d copies (%.0f MB)" % (n_lg, n_lg * ubytes / 1e6)}
         del ug, lgs
 
