@@ -85,6 +85,7 @@ struct tt_plan_s {
   int kernel = TT_KERNEL_MMA_SYNC;
   int C = 1;
   int C_paged = 1;   // ranges of paged calls (differs from C on 2-SM plans)
+  int C_decode = 1;  // ranges of contiguous decode calls
   int key_tile = 64;
   int variant = 0;
   int R = 0, g = 1;
@@ -331,6 +332,15 @@ tt_status_t tt_block_attn_plan(const tt_block_attn_desc* desc, int device, tt_pl
     P->causal_T = (long long)d.batch * d.num_kv_heads * acc;
   }
 
+  // Decode calls on the default tcgen05 kernel: with U = batch * Hkv units and at least two
+  // ranges per unit, U * floor(SMs / U) ranges put every unit boundary on a range boundary when
+  // the context lengths are equal, so no range carries a second segment (its extra Q load and
+  // partial epilogue) at the cost of fewer than U idle SMs.  Ragged lengths are split as before.
+  P->C_decode = P->C;
+  if (P->kernel == TT_KERNEL_TCGEN05 && P->variant == 0 && d.num_ctas <= 0) {
+    const long long U = (long long)d.batch * d.num_kv_heads;
+    if (U > 0 && P->sm_count / U >= 2) P->C_decode = (int)(U * (P->sm_count / U));
+  }
   // scratch layout (256-byte aligned pieces).  A 2-SM plan runs one range per SM pair, but
   // its paged calls run on the one-CTA-per-SM kernel: room for one range per SM as well.
   P->C_paged = (P->kernel == TT_KERNEL_TCGEN05 && P->variant == 3 && d.num_ctas <= 0) ? P->sm_count : P->C;
@@ -426,6 +436,7 @@ tt_status_t tt_block_attn(tt_plan_t plan, const void* q, const void* k_ctx, cons
     return fail(TT_ERR_INVALID_ARG, "tensor pointer not 16-byte aligned");
   DeviceGuard guard(plan->device);
   tt::Problem p = base_problem(plan);
+  p.C = plan->C_decode;
   p.mode = tt::kDecode;
   p.NB = 1;
   p.ctx_stride = d.ctx_capacity;
@@ -465,7 +476,7 @@ tt_status_t tt_block_attn_paged(tt_plan_t plan, const void* q, const void* k_pag
   p.mode = tt::kDecode;
   p.NB = 1;
   p.variant = 0;  // the paged loads live in the default tcgen05 kernel (and the mma.sync one)
-  p.C = plan->C_paged;
+  p.C = plan->variant == 3 ? plan->C_paged : plan->C_decode;
   p.ctx_stride = pages_per_seq * page_size;
   int shift = 0;
   while ((1 << shift) < page_size) ++shift;
