@@ -11,13 +11,15 @@
 // key tile is read from HBM once and feeds up to 256 query rows.
 //
 // Roles (384 threads):
-//   warp 0       TMA producer: Q of each segment, then K and V tiles of every
-//                key tile into a ring of shared-memory slots (128-byte swizzle);
-//                for a tile whose valid rows are not a multiple of 16 it zeroes
-//                the V rows the last MMA k-step would otherwise read.
-//   warp 1       TMEM owner; lane 0 issues the MMAs of M-tile 0: S = Q_0 K^T into
-//                TMEM, O_0 += P V with P read from TMEM (aliasing its S buffer)
-//   warp 2       lane 0 issues the MMAs of M-tile 1 (when the unit has two)
+//   warp 0       TMA producer of Q (each segment) and of the K tiles, into the K half
+//                of a ring of shared-memory slots (128-byte swizzle)
+//   warp 3       TMA producer of the V tiles, into the V half of the ring; for a
+//                tile whose valid rows are not a multiple of 16 it zeroes the V rows
+//                the last MMA k-step would otherwise read
+//   warp 1       TMEM owner; issues the MMAs of M-tile 0 (one elected lane): S =
+//                Q_0 K^T into TMEM, O_0 += P V with P read from TMEM (aliasing its S
+//                buffer)
+//   warp 2       issues the MMAs of M-tile 1 (when the unit has two)
 //   warps 4..7   softmax warpgroup of M-tile 0 (thread = TMEM lane = row)
 //   warps 8..11  softmax warpgroup of M-tile 1
 // TMEM columns: M-tile m owns S buffers [128m, 128m+128) (NBUF buffers of NK
@@ -51,10 +53,10 @@ constexpr int kMaxRows = 256;
 constexpr int kRowBytes = 128;              // one 64-element bf16 row of a swizzled half
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
 
-template <int D, int NK>
+template <int D, int NK, bool QT>
 struct Cfg {
   static constexpr int kHalves = D / 64;
-  static constexpr int kBufs = 128 / NK;                       // S buffers per M-tile
+  static constexpr int kBufs = QT ? 1 : 128 / NK;              // S buffers per M-tile
   static constexpr int kSlotBytes = NK * kRowBytes * kHalves;  // one K or V tile
   static constexpr int kStages = (128 * 1024) / kSlotBytes;    // 128 KB ring
   static constexpr int kQBytes = kMaxRows * kRowBytes * kHalves;
@@ -75,6 +77,8 @@ struct Bars {
   uint64_t q_full, q_empty, tail, drain;
   uint64_t s_full[2][2], p_full[2][2];  // [M-tile][S buffer]
   uint64_t pv_done[2], o_full[2], o_empty[2];
+  uint64_t qt_full[2];                  // Q rows of M-tile m copied into TMEM (QT form)
+  uint64_t turn[2];                     // QT form with two M-tiles: softmax warpgroup m may start a tile
   uint64_t kv_full[16], kv_empty[16];
 };
 
@@ -142,10 +146,11 @@ __device__ __forceinline__ void fused_combine(const Problem& p, uint8_t* scratch
   }
 }
 
-template <int D, int NK>
+template <int D, int NK, bool QT>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tcgen05_kernel(const Problem p, const __grid_constant__ TmaMaps maps) {
-  using C = Cfg<D, NK>;
+  using C = Cfg<D, NK, QT>;
+  static_assert(!QT || NK == 64, "the Q-in-TMEM form runs 64-key tiles");
   constexpr int NBUF = C::kBufs;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -172,7 +177,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (tid == 0) {
     mbar_init(smem_u32(&bars->q_full), 1);
-    mbar_init(smem_u32(&bars->q_empty), MT);  // one commit per M-tile issuer
+    // one commit per M-tile issuer; in the QT form one arrival per softmax thread (its row copied)
+    mbar_init(smem_u32(&bars->q_empty), QT ? MT * 128 : MT);
     mbar_init(smem_u32(&bars->tail), 1);
     mbar_init(smem_u32(&bars->drain), MT);
     for (int m = 0; m < 2; ++m) {
@@ -181,6 +187,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(smem_u32(&bars->p_full[m][b]), 128);
       }
       mbar_init(smem_u32(&bars->pv_done[m]), 1);
+      mbar_init(smem_u32(&bars->qt_full[m]), 128);
+      mbar_init(smem_u32(&bars->turn[m]), 128);
       mbar_init(smem_u32(&bars->o_full[m]), 1);
       mbar_init(smem_u32(&bars->o_empty[m]), 128);
     }
@@ -225,22 +233,31 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (have_work && warp < 4) regs_dec<C::kCtrlRegs>();
   }
 
-  if (warp == 0 && have_work) {
-    // ============================================================ producer ==
-    uint32_t it = 0, q_it = 0, tail_ph = 0;
+  if ((warp == 0 || warp == 3) && have_work) {
+    // =========================================================== producers ==
+    // Warp 0 loads Q of each segment and the K tiles, warp 3 the V tiles, each into its own
+    // half of the ring: K(t) of the CTA's t-th tile in stage t % H, V(t) in stage H + t % H
+    // (H = half the stages).  A K slot frees as soon as both M-tiles' S MMAs have read it, long
+    // before P V frees the V slot of the same tile, so K loads run further ahead than they
+    // could behind V loads in one ring.
+    constexpr int H = C::kStages / 2;
+    const int kv = warp == 0 ? 0 : 1;
+    uint32_t t = 0, q_it = 0, tail_ph = 0;
     bool ok = true;
     Unit x = sh->first;
     for (; ok;) {
       const Segment sg = segment_of(x, start, end, c);
-      ok = mbar_wait(smem_u32(&bars->q_empty), (q_it & 1) ^ 1, wc);
-      if (!ok) break;
-      if (lane == 0) {
-        const uint32_t bar = smem_u32(&bars->q_full);
-        mbar_arrive_expect_tx(bar, (uint32_t)(p.R * kRowBytes * C::kHalves));
-        for (int hf = 0; hf < C::kHalves; ++hf)
-          tma_load_3d(q_s + hf * (kMaxRows * kRowBytes), &maps.q, bar, hf * 64, x.h * p.g, x.ns * p.S);
+      if (kv == 0) {
+        ok = mbar_wait(smem_u32(&bars->q_empty), (q_it & 1) ^ 1, wc);
+        if (!ok) break;
+        if (lane == 0) {
+          const uint32_t bar = smem_u32(&bars->q_full);
+          mbar_arrive_expect_tx(bar, (uint32_t)(p.R * kRowBytes * C::kHalves));
+          for (int hf = 0; hf < C::kHalves; ++hf)
+            tma_load_3d(q_s + hf * (kMaxRows * kRowBytes), &maps.q, bar, hf * 64, x.h * p.g, x.ns * p.S);
+        }
+        ++q_it;
       }
-      ++q_it;
       const int ctx_row0 = (x.n * p.Hkv + x.h) * p.ctx_stride;
       // paged cache: a context tile is loaded in slices of psub rows, one per page (pages of
       // at least NK keys hold whole tiles); slices past the tile's last key are not loaded
@@ -254,55 +271,53 @@ __global__ void __launch_bounds__(kThreads, 1)
         return row < 0 ? (p.num_pages * p.Hkv) << p.page_shift : row;  // a bad page reads as zeros
       };
       int cur_row = slice_row(sg.lo);
-      for (int i = sg.lo; i < sg.hi && ok; ++i) {
+      for (int i = sg.lo; i < sg.hi && ok; ++i, ++t) {
         const TileKeys tk = tile_keys(p, x, i);
         const int box_rows = tk.is_blk ? min(p.S, NK) : (p.page_table ? ceil_div(tk.count, psub) * psub : NK);
         const uint32_t bytes = (uint32_t)(box_rows * kRowBytes * C::kHalves);
         const int nsl = p.page_table && !tk.is_blk ? box_rows / psub : 0;   // slices of a paged tile
         const int row_i = cur_row;
         if (i + 1 < sg.hi) cur_row = slice_row(i + 1);
-        for (int kv = 0; kv < 2 && ok; ++kv, ++it) {
-          const int s = it % C::kStages;
-          ok = mbar_wait(smem_u32(&bars->kv_empty[s]), ((it / C::kStages) & 1) ^ 1, wc);
+        const int s = kv * H + (int)(t % H);
+        ok = mbar_wait(smem_u32(&bars->kv_empty[s]), ((t / H) & 1) ^ 1, wc);
+        if (!ok) break;
+        const uint32_t slot = kv_s + s * C::kSlotBytes;
+        const CUtensorMap* m = tk.is_blk ? (kv ? &maps.v_blk : &maps.k_blk) : (kv ? &maps.v_ctx : &maps.k_ctx);
+        // V rows [count, round16(count)) are read by the last PV k-step: zero them.
+        const bool fix = kv == 1 && (tk.count & 15) != 0;
+        const uint32_t bar = fix ? smem_u32(&bars->tail) : smem_u32(&bars->kv_full[s]);
+        if (lane == 0) mbar_arrive_expect_tx(bar, bytes);
+        if (nsl > 0) {
+          // each slice lands at its row offset in the stage (a multiple of 2 KB: the swizzle
+          // pattern stays aligned); issued after the expected byte count is set
+          __syncwarp();
+          if (lane < nsl)
+            for (int hf = 0; hf < C::kHalves; ++hf)
+              tma_load_2d(slot + hf * (NK * kRowBytes) + lane * psub * kRowBytes, m, bar, hf * 64, row_i);
+        } else if (lane == 0) {
+          for (int hf = 0; hf < C::kHalves; ++hf) {
+            const uint32_t dst = slot + hf * (NK * kRowBytes);
+            if (tk.is_blk) tma_load_3d(dst, m, bar, hf * 64, x.h, x.ns * p.S + tk.first);
+            else tma_load_2d(dst, m, bar, hf * 64, ctx_row0 + tk.first);
+          }
+        }
+        if (fix) {
+          ok = mbar_wait(smem_u32(&bars->tail), tail_ph, wc);
+          tail_ph ^= 1;
           if (!ok) break;
-          const uint32_t slot = kv_s + s * C::kSlotBytes;
-          const CUtensorMap* m = tk.is_blk ? (kv ? &maps.v_blk : &maps.k_blk) : (kv ? &maps.v_ctx : &maps.k_ctx);
-          // V rows [count, round16(count)) are read by the last PV k-step: zero them.
-          const bool fix = kv == 1 && (tk.count & 15) != 0;
-          const uint32_t bar = fix ? smem_u32(&bars->tail) : smem_u32(&bars->kv_full[s]);
-          if (lane == 0) mbar_arrive_expect_tx(bar, bytes);
-          if (nsl > 0) {
-            // each slice lands at its row offset in the stage (a multiple of 2 KB: the swizzle
-            // pattern stays aligned); issued after the expected byte count is set
-            __syncwarp();
-            if (lane < nsl)
-              for (int hf = 0; hf < C::kHalves; ++hf)
-                tma_load_2d(slot + hf * (NK * kRowBytes) + lane * psub * kRowBytes, m, bar, hf * 64, row_i);
-          } else if (lane == 0) {
-            for (int hf = 0; hf < C::kHalves; ++hf) {
-              const uint32_t dst = slot + hf * (NK * kRowBytes);
-              if (tk.is_blk) tma_load_3d(dst, m, bar, hf * 64, x.h, x.ns * p.S + tk.first);
-              else tma_load_2d(dst, m, bar, hf * 64, ctx_row0 + tk.first);
-            }
+          const int r0 = tk.count, r1 = round16(tk.count);
+          const int n16 = (r1 - r0) * 8 * C::kHalves;  // 16-byte chunks to clear
+          for (int e = lane; e < n16; e += 32) {
+            const int hf = e / ((r1 - r0) * 8);
+            const int rem = e - hf * (r1 - r0) * 8;
+            const int row = r0 + rem / 8, ch = rem % 8;
+            uint4* dst = reinterpret_cast<uint4*>(smem + C::kStageOff + s * C::kSlotBytes +
+                                                  hf * (NK * kRowBytes) + row * kRowBytes + ch * 16);
+            *dst = make_uint4(0, 0, 0, 0);
           }
-          if (fix) {
-            ok = mbar_wait(smem_u32(&bars->tail), tail_ph, wc);
-            tail_ph ^= 1;
-            if (!ok) break;
-            const int r0 = tk.count, r1 = round16(tk.count);
-            const int n16 = (r1 - r0) * 8 * C::kHalves;  // 16-byte chunks to clear
-            for (int e = lane; e < n16; e += 32) {
-              const int hf = e / ((r1 - r0) * 8);
-              const int rem = e - hf * (r1 - r0) * 8;
-              const int row = r0 + rem / 8, ch = rem % 8;
-              uint4* dst = reinterpret_cast<uint4*>(smem + C::kStageOff + s * C::kSlotBytes +
-                                                    hf * (NK * kRowBytes) + row * kRowBytes + ch * 16);
-              *dst = make_uint4(0, 0, 0, 0);
-            }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&bars->kv_full[s]));
-          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(&bars->kv_full[s]));
         }
       }
       if (!ok || sg.last) break;
@@ -312,70 +327,81 @@ __global__ void __launch_bounds__(kThreads, 1)
       // drain: wait (briefly) for loads that may still be landing in shared memory
       int dummy = 0;
       WaitCtx dw{&dummy, nullptr, 2000000ull};
-      for (uint32_t j = (it > (uint32_t)C::kStages ? it - C::kStages : 0); j < it; ++j)
-        mbar_wait(smem_u32(&bars->kv_full[j % C::kStages]), (j / C::kStages) & 1, dw);
+      for (uint32_t j = (t > (uint32_t)H ? t - H : 0); j < t; ++j)
+        mbar_wait(smem_u32(&bars->kv_full[kv * H + j % H]), (j / H) & 1, dw);
       if (q_it) mbar_wait(smem_u32(&bars->q_full), (q_it - 1) & 1, dw);
     }
   } else if ((warp == 1 || (warp == 2 && MT == 2)) && have_work) {
     // ====================================================== MMA issuers ==
-    // One thread per M-tile (warp 1 lane 0: M-tile 0, warp 2 lane 0: M-tile 1), so an M-tile
-    // whose P is not ready never holds back the other's MMAs; the tensor core interleaves the
-    // two instruction streams.  Each thread commits its own reads of a ring slot and of Q,
-    // and those barriers expect one commit per M-tile.
-    if (lane == 0) {
-      const int m = warp - 1;
-      uint32_t it = 0, q_it = 0, G = 0, seg_cnt = 0;
-      bool ok = true;
-      Unit x = sh->first;
-      // descriptors: a start-address offset is added in 16-byte units to the low field
-      const uint64_t qdesc = smem_desc_sw128(q_s + m * 128 * kRowBytes, 16, 1024);
-      const uint64_t kdesc0 = smem_desc_sw128(kv_s, 16, 1024);
-      const uint64_t vdesc0 = smem_desc_sw128(kv_s, NK * kRowBytes, 1024);
-      const uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
-      const uint32_t idesc_s0 = idesc_bf16_f32(128, 0, 0, 0);
-      const uint32_t s_tmem = tmem + m * 128, o_tmem = tmem + 256 + m * D;
-      auto issue_s = [&](int buf, uint32_t slot, int n_mma) {
-        const uint32_t idesc = idesc_s0 | ((uint32_t)(n_mma >> 3) << 17);
-        const uint64_t kd = kdesc0 + (uint64_t)((slot * C::kSlotBytes) >> 4);
+    // One warp per M-tile (warp 1: M-tile 0, warp 2: M-tile 1), so an M-tile whose P is not
+    // ready never holds back the other's MMAs; the tensor core interleaves the two instruction
+    // streams.  The whole warp runs the control flow (waits, tile bookkeeping, descriptors stay
+    // warp-uniform) and one elected lane issues each burst of MMAs and its commits.  Each warp
+    // commits its own reads of a ring slot and of Q, and those barriers expect one commit per
+    // M-tile.
+    const int m = warp - 1;
+    constexpr int H = C::kStages / 2;   // K tiles in stages [0, H), V tiles in [H, 2H)
+    uint32_t tb = 0, q_it = 0, G = 0, seg_cnt = 0;   // tb: the CTA's tile count before this segment
+    bool ok = true;
+    Unit x = sh->first;
+    // descriptors: a start-address offset is added in 16-byte units to the low field
+    const uint64_t qdesc = smem_desc_sw128(q_s + m * 128 * kRowBytes, 16, 1024);
+    const uint64_t kdesc0 = smem_desc_sw128(kv_s, 16, 1024);
+    const uint64_t vdesc0 = smem_desc_sw128(kv_s, NK * kRowBytes, 1024);
+    const uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
+    const uint32_t idesc_s0 = idesc_bf16_f32(128, 0, 0, 0);
+    const uint32_t s_tmem = tmem + m * (QT ? 64 : 128), o_tmem = tmem + 256 + m * D;
+    const uint32_t q_tmem = tmem + 128 + m * 64;   // QT form: Q_m as bf16 pairs, D / 2 columns
+    // S = Q K^T of one tile into buffer `buf` (K in ring slot `slot`), then its commits
+    auto issue_s = [&](int buf, uint32_t slot, int n_mma) {
+      const uint32_t idesc = idesc_s0 | ((uint32_t)(n_mma >> 3) << 17);
+      const uint64_t kd = kdesc0 + (uint64_t)((slot * C::kSlotBytes) >> 4);
+      if (elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * (kMaxRows * kRowBytes) + (kk & 3) * 32;
           const uint32_t koff = (kk >> 2) * (NK * kRowBytes) + (kk & 3) * 32;
-          tc_mma_ss(s_tmem + buf * NK, qdesc + (off >> 4), kd + (koff >> 4), idesc, kk > 0);
+          if constexpr (QT)
+            tc_mma_ts(s_tmem + buf * NK, q_tmem + kk * 8, kd + (koff >> 4), idesc, kk > 0);
+          else
+            tc_mma_ss(s_tmem + buf * NK, qdesc + (off >> 4), kd + (koff >> 4), idesc, kk > 0);
         }
-      };
-      auto kv_wait = [&](uint32_t e) {
-        return mbar_wait(smem_u32(&bars->kv_full[e % C::kStages]), (e / C::kStages) & 1, wc);
-      };
-      for (; ok;) {
-        const Segment sg = segment_of(x, start, end, c);
-        const int n = sg.hi - sg.lo;
-        ok = mbar_wait(smem_u32(&bars->q_full), q_it & 1, wc);
-        ++q_it;
+        tc_commit(smem_u32(&bars->s_full[m][buf]));
+        tc_commit(smem_u32(&bars->kv_empty[slot]));
+      }
+      __syncwarp();
+    };
+    // K (kv = 0) or V (kv = 1) of the CTA's tile t
+    auto kv_wait = [&](uint32_t t, int kv) {
+      return mbar_wait_warp(smem_u32(&bars->kv_full[kv * H + t % H]), (t / H) & 1, wc);
+    };
+    for (; ok;) {
+      const Segment sg = segment_of(x, start, end, c);
+      const int n = sg.hi - sg.lo;
+      if constexpr (QT) ok = mbar_wait_warp(smem_u32(&bars->qt_full[m]), seg_cnt & 1, wc);
+      else ok = mbar_wait_warp(smem_u32(&bars->q_full), q_it & 1, wc);
+      ++q_it;
+      if (!ok) break;
+      tc_fence_after();
+      // prologue: S of the segment's first NBUF tiles
+      for (int j = 0; j < NBUF && j < n && ok; ++j) {
+        ok = kv_wait(tb + j, 0);
         if (!ok) break;
         tc_fence_after();
-        // prologue: S of the segment's first NBUF tiles (K of tile j = ring entry it + 2j)
-        for (int j = 0; j < NBUF && j < n && ok; ++j) {
-          ok = kv_wait(it + 2 * j);
-          if (!ok) break;
-          tc_fence_after();
-          const int nk = round16(tile_keys(p, x, sg.lo + j).count);
-          const uint32_t ks = (it + 2 * j) % C::kStages;
-          issue_s((G + j) % NBUF, ks, nk);
-          tc_commit(smem_u32(&bars->s_full[m][(G + j) % NBUF]));
-          tc_commit(smem_u32(&bars->kv_empty[ks]));
-        }
-        for (int j = 0; j < n && ok; ++j, ++G) {
-          const int b = G % NBUF;
-          const uint32_t ev = it + 2 * j + 1;  // V of tile j
-          ok = kv_wait(ev);
-          if (ok) ok = mbar_wait(smem_u32(&bars->p_full[m][b]), (G / NBUF) & 1, wc);
-          if (ok && j == 0) ok = mbar_wait(smem_u32(&bars->o_empty[m]), (seg_cnt & 1) ^ 1, wc);
-          if (!ok) break;
-          tc_fence_after();
-          const int nv = round16(tile_keys(p, x, sg.lo + j).count);
-          const uint64_t vd = vdesc0 + (uint64_t)(((ev % C::kStages) * C::kSlotBytes) >> 4);
-          const uint32_t pa = s_tmem + b * NK;
+        issue_s((G + j) % NBUF, (tb + j) % H, round16(tile_keys(p, x, sg.lo + j).count));
+      }
+      for (int j = 0; j < n && ok; ++j, ++G) {
+        const int b = G % NBUF;
+        const uint32_t ev = H + (tb + j) % H;  // stage of V of tile j
+        ok = kv_wait(tb + j, 1);
+        if (ok) ok = mbar_wait_warp(smem_u32(&bars->p_full[m][b]), (G / NBUF) & 1, wc);
+        if (ok && j == 0) ok = mbar_wait_warp(smem_u32(&bars->o_empty[m]), (seg_cnt & 1) ^ 1, wc);
+        if (!ok) break;
+        tc_fence_after();
+        const int nv = round16(tile_keys(p, x, sg.lo + j).count);
+        const uint64_t vd = vdesc0 + (uint64_t)((ev * C::kSlotBytes) >> 4);
+        const uint32_t pa = s_tmem + b * NK;
+        if (elect_one()) {
           if (nv == NK) {
 #pragma unroll
             for (int kk = 0; kk < NK / 16; ++kk)
@@ -387,32 +413,34 @@ __global__ void __launch_bounds__(kThreads, 1)
                         (j > 0 || kk > 0) ? 1u : 0u);
           }
           tc_commit(smem_u32(&bars->pv_done[m]));
-          tc_commit(smem_u32(&bars->kv_empty[ev % C::kStages]));
-          if (j + NBUF < n) {
-            // S of tile j + NBUF into buffer b, after P V(j) has read P(j) from it (in issue order)
-            const uint32_t ek = it + 2 * (j + NBUF);
-            ok = kv_wait(ek);
-            if (!ok) break;
-            tc_fence_after();
-            issue_s(b, ek % C::kStages, round16(tile_keys(p, x, sg.lo + j + NBUF).count));
-            tc_commit(smem_u32(&bars->s_full[m][b]));
-            tc_commit(smem_u32(&bars->kv_empty[ek % C::kStages]));
-          }
+          tc_commit(smem_u32(&bars->kv_empty[ev]));
         }
-        if (!ok) break;
-        it += 2 * n;
-        tc_commit(smem_u32(&bars->o_full[m]));
-        tc_commit(smem_u32(&bars->q_empty));
-        ++seg_cnt;
-        if (sg.last) break;
-        x = make_unit(p, x.u + 1, x.Tu + x.tiles);
+        __syncwarp();
+        if (j + NBUF < n) {
+          // S of tile j + NBUF into buffer b, after P V(j) has read P(j) from it (in issue order)
+          ok = kv_wait(tb + j + NBUF, 0);
+          if (!ok) break;
+          tc_fence_after();
+          issue_s(b, (tb + j + NBUF) % H, round16(tile_keys(p, x, sg.lo + j + NBUF).count));
+        }
       }
-      // drain every MMA this thread issued before TMEM can be released
-      tc_commit(smem_u32(&bars->drain));
-      int dummy = 0;
-      WaitCtx dw{&dummy, nullptr, 2000000ull};
-      mbar_wait(smem_u32(&bars->drain), 0, dw);
+      if (!ok) break;
+      tb += n;
+      if (elect_one()) {
+        tc_commit(smem_u32(&bars->o_full[m]));
+        if constexpr (!QT) tc_commit(smem_u32(&bars->q_empty));
+      }
+      __syncwarp();
+      ++seg_cnt;
+      if (sg.last) break;
+      x = make_unit(p, x.u + 1, x.Tu + x.tiles);
     }
+    // drain every MMA this warp issued before TMEM can be released
+    if (elect_one()) tc_commit(smem_u32(&bars->drain));
+    __syncwarp();
+    int dummy = 0;
+    WaitCtx dw{&dummy, nullptr, 2000000ull};
+    mbar_wait(smem_u32(&bars->drain), 0, dw);
     __syncwarp();
   } else if (warp >= 4 && have_work) {
     // ========================================================= softmax WGs ==
@@ -423,12 +451,40 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r = m * 128 + row;         // packed row of the unit
     if (m < MT) {
       const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
-      const uint32_t s_base = tmem + lane_off + m * 128;  // + buffer * NK
+      const uint32_t s_base = tmem + lane_off + m * (QT ? 64 : 128);  // + buffer * NK
       const uint32_t o_addr = tmem + lane_off + 256 + m * D;
       float* stage = epi + (warp - 4) * 32 * 32;
-      uint32_t G = 0, seg_cnt = 0;
+      uint32_t G = 0, seg_cnt = 0, q_it = 0;
       bool ok = true;
       Unit x = sh->first;
+      // QT form: this thread's Q row (row r of the 128-byte-swizzled shared tile) into TMEM lane
+      // `row` of Q_m, then the shared tile is released.  Called once the M-tile's S MMAs of the
+      // previous segment have all completed (its last S was consumed), so Q_m is free.
+      auto copy_q = [&]() -> bool {
+        if (!mbar_wait(smem_u32(&bars->q_full), q_it & 1, wc)) return false;
+        ++q_it;
+        const uint32_t q_addr = tmem + lane_off + 128 + m * 64;
+#pragma unroll
+        for (int hf = 0; hf < C::kHalves; ++hf) {
+          uint32_t v[32];
+#pragma unroll
+          for (int cq = 0; cq < 8; ++cq) {
+            const uint4 u = *reinterpret_cast<const uint4*>(smem + hf * (kMaxRows * kRowBytes) + r * kRowBytes +
+                                                            ((cq ^ (r & 7)) << 4));
+            v[4 * cq] = u.x;
+            v[4 * cq + 1] = u.y;
+            v[4 * cq + 2] = u.z;
+            v[4 * cq + 3] = u.w;
+          }
+          tmem_st32(q_addr + 32 * hf, v);
+        }
+        tc_wait_st();
+        tc_fence_before();
+        mbar_arrive(smem_u32(&bars->qt_full[m]));
+        mbar_arrive(smem_u32(&bars->q_empty));
+        return true;
+      };
+      if constexpr (QT) ok = copy_q();
       for (; ok;) {
         const Segment sg = segment_of(x, start, end, c);
         float m_ref = -INFINITY, l = 0.f;
@@ -476,6 +532,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int b = G % NBUF;
           const uint32_t s_addr = s_base + b * NK;
           ok = mbar_wait(smem_u32(&bars->s_full[m][b]), (G / NBUF) & 1, wc);
+          // QT form, two M-tiles: the warpgroups take turns tile by tile (M-tile 0 first), so one
+          // softmax runs while the other M-tile's P V and next S occupy the tensor core
+          if constexpr (QT) {
+            if (ok && MT == 2 && (m == 1 || G > 0))
+              ok = mbar_wait(smem_u32(&bars->turn[m]), (m == 1 ? G : G - 1) & 1, wc);
+          }
           if (!ok) break;
           tc_fence_after();
           // (128-key tiles keep a single masked path: a second copy of their 128-register body
@@ -486,11 +548,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = count == NK ? tile(std::true_type{}, count, s_addr, i == sg.lo)
                              : tile(std::false_type{}, count, s_addr, i == sg.lo);
           if (!ok) break;
+          if constexpr (QT) {
+            if (MT == 2) mbar_arrive(smem_u32(&bars->turn[m ^ 1]));
+          }
           tc_wait_st();
           tc_fence_before();
           mbar_arrive(smem_u32(&bars->p_full[m][b]));
         }
         if (!ok) break;
+        // QT form: the next segment's Q goes into TMEM before this epilogue, so its first S
+        // MMAs overlap the epilogue
+        if constexpr (QT) {
+          if (!sg.last && !copy_q()) break;
+        }
         // ---- epilogue: O / l to the output (or the segment's partial) ----
         ok = mbar_wait(smem_u32(&bars->o_full[m]), seg_cnt & 1, wc);
         if (!ok) break;
@@ -562,30 +632,30 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (p.grid_bar != nullptr) fused_combine<D>(p, smem + C::kEpiOff, *(volatile int*)&sh->abort_flag != 0);
 }
 
-template <int D, int NK>
+template <int D, int NK, bool QT>
 void set_smem_attr() {
-  cudaFuncSetAttribute(attn_tcgen05_kernel<D, NK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                       Cfg<D, NK>::kSmemBytes);
+  cudaFuncSetAttribute(attn_tcgen05_kernel<D, NK, QT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       Cfg<D, NK, QT>::kSmemBytes);
 }
 
-template <int D, int NK>
+template <int D, int NK, bool QT = false>
 cudaError_t launch(const Problem& p, const TmaMaps& maps, cudaStream_t stream) {
   if (p.grid_bar == nullptr) {
-    attn_tcgen05_kernel<D, NK><<<p.C, kThreads, Cfg<D, NK>::kSmemBytes, stream>>>(p, maps);
+    attn_tcgen05_kernel<D, NK, QT><<<p.C, kThreads, Cfg<D, NK, QT>::kSmemBytes, stream>>>(p, maps);
     return cudaGetLastError();
   }
   // cooperative: every CTA must be resident at once for the grid barrier of the fused combine
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.C, 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = Cfg<D, NK>::kSmemBytes;
+  cfg.dynamicSmemBytes = Cfg<D, NK, QT>::kSmemBytes;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeCooperative;
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, attn_tcgen05_kernel<D, NK>, p, maps);
+  return cudaLaunchKernelEx(&cfg, attn_tcgen05_kernel<D, NK, QT>, p, maps);
 }
 
 }  // namespace
@@ -594,16 +664,21 @@ bool tcgen05_key_tile_supported(int key_tile) { return key_tile == 64 || key_til
 
 cudaError_t launch_attn_tcgen05(const Problem& p, const TmaMaps& maps, cudaStream_t stream) {
   static const bool attr_done = [] {
-    set_smem_attr<128, 128>();
-    set_smem_attr<128, 64>();
-    set_smem_attr<64, 128>();
-    set_smem_attr<64, 64>();
+    set_smem_attr<128, 128, false>();
+    set_smem_attr<128, 64, false>();
+    set_smem_attr<64, 128, false>();
+    set_smem_attr<64, 64, false>();
+    set_smem_attr<128, 64, true>();
+    set_smem_attr<64, 64, true>();
     return true;
   }();
   (void)attr_done;
   if (!tcgen05_key_tile_supported(p.key_tile)) return cudaErrorInvalidValue;
   // variant 2: head_dim 128 with 128-key tiles on the transposed-PV kernel (attn_tcgen05_pt.cu)
   if (p.D == 128 && p.key_tile == 128 && p.variant == 2) return launch_attn_pt(p, maps, stream);
+  // variant 1: 64-key tiles with Q in TMEM (the S MMAs read only K from shared memory)
+  if (p.variant == 1 && p.key_tile == 64)
+    return p.D == 128 ? launch<128, 64, true>(p, maps, stream) : launch<64, 64, true>(p, maps, stream);
   if (p.D == 128) return p.key_tile == 128 ? launch<128, 128>(p, maps, stream) : launch<128, 64>(p, maps, stream);
   return p.key_tile == 128 ? launch<64, 128>(p, maps, stream) : launch<64, 64>(p, maps, stream);
 }
