@@ -14,7 +14,7 @@
 //   warp 0       TMA producer: Q and dO of the item, then K and V of its key tiles
 //                (tile 0 = the block's own keys, tiles 1.. = its visible context, 64
 //                keys each) into a ring of shared-memory slots (128-byte swizzle)
-//   warp 1       TMEM owner and MMA issuer (one thread):
+//   warp 1       TMEM owner and MMA issuer (one elected lane issues):
 //                  S(j) = Q K(j)^T and dP(j) = dO V(j)^T into TMEM buffer j % 2 with Q
 //                  and dO read from TMEM (A operands), K and V from shared memory,
 //                  dQ += dS(j) K(j) with dS read from TMEM as a bf16 pair hi + lo
@@ -244,20 +244,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ============================================================= MMA warp ==
-    if (lane == 0) {
-      uint32_t it_kv = 0, q_it = 0, G = 0, item_cnt = 0;
-      bool ok = true;
-      const uint32_t q_tmem = tmem + 384, o_tmem = tmem + 448;
-      const uint64_t kdesc0 = smem_desc_sw128(kv_s, 16, 1024);              // K-major (S, dP)
-      const uint64_t kmn0 = smem_desc_sw128(kv_s, kNK * kRowBytes, 1024);   // MN-major (dQ)
-      const uint32_t idesc_sd0 = idesc_bf16_f32(128, 0, 0, 0);   // A (Q, dO) from TMEM, K-major B
-      const uint32_t idesc_dq = idesc_bf16_f32(128, D, 0, 1);
-      const uint32_t dq_tmem = tmem + 256;
-      // S = Q K^T and dP = dO V^T of tile j into buffer b (K, V = ring entries ek, ek + 1)
-      auto issue_sd = [&](int b, uint32_t ek, int nk) {
-        const uint32_t idesc = idesc_sd0 | ((uint32_t)(nk >> 3) << 17);
-        const uint64_t kd = kdesc0 + (uint64_t)(((ek % kStages) * C::kSlotBytes) >> 4);
-        const uint64_t vd = kdesc0 + (uint64_t)((((ek + 1) % kStages) * C::kSlotBytes) >> 4);
+    // The whole warp runs the control flow (waits and descriptors stay warp-uniform); one
+    // elected lane issues each burst of MMAs and its commits.
+    uint32_t it_kv = 0, q_it = 0, G = 0, item_cnt = 0;
+    bool ok = true;
+    const uint32_t q_tmem = tmem + 384, o_tmem = tmem + 448;
+    const uint64_t kdesc0 = smem_desc_sw128(kv_s, 16, 1024);              // K-major (S, dP)
+    const uint64_t kmn0 = smem_desc_sw128(kv_s, kNK * kRowBytes, 1024);   // MN-major (dQ)
+    const uint32_t idesc_sd0 = idesc_bf16_f32(128, 0, 0, 0);   // A (Q, dO) from TMEM, K-major B
+    const uint32_t idesc_dq = idesc_bf16_f32(128, D, 0, 1);
+    const uint32_t dq_tmem = tmem + 256;
+    // S = Q K^T and dP = dO V^T of tile j into buffer b (K, V = ring entries ek, ek + 1), then
+    // the commits: S and dP ready, V read
+    auto issue_sd = [&](int b, uint32_t ek, int nk) {
+      const uint32_t idesc = idesc_sd0 | ((uint32_t)(nk >> 3) << 17);
+      const uint64_t kd = kdesc0 + (uint64_t)(((ek % kStages) * C::kSlotBytes) >> 4);
+      const uint64_t vd = kdesc0 + (uint64_t)((((ek + 1) % kStages) * C::kSlotBytes) >> 4);
+      if (elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t koff = (kk >> 2) * (kNK * kRowBytes) + (kk & 3) * 32;
@@ -268,71 +271,86 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t koff = (kk >> 2) * (kNK * kRowBytes) + (kk & 3) * 32;
           tc_mma_ts(tmem + 128 + 64 * b, o_tmem + kk * 8, vd + (koff >> 4), idesc, kk > 0);
         }
-      };
-      auto kv_wait = [&](uint32_t e) {
-        return mbar_wait(smem_u32(&bars->kv_full[e % kStages]), (e / kStages) & 1, wc);
-      };
-      for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x, ++item_cnt) {
-        const Item x = item_of(p, idx, MT);
-        const int n = x.tiles;
-        ok = mbar_wait(smem_u32(&bars->qo_full), q_it & 1, wc);
-        ++q_it;
+        tc_commit(smem_u32(&bars->sd_full[b]));
+        tc_commit(smem_u32(&bars->kv_empty[(ek + 1) % kStages]));   // V read by dP
+      }
+      __syncwarp();
+    };
+    auto kv_wait = [&](uint32_t e) {
+      return mbar_wait_warp(smem_u32(&bars->kv_full[e % kStages]), (e / kStages) & 1, wc);
+    };
+    for (int idx = blockIdx.x; idx < n_items && ok; idx += gridDim.x, ++item_cnt) {
+      const Item x = item_of(p, idx, MT);
+      const int n = x.tiles;
+      ok = mbar_wait_warp(smem_u32(&bars->qo_full), q_it & 1, wc);
+      ++q_it;
+      if (!ok) break;
+      tc_fence_after();
+      // prologue: S and dP of the first two tiles
+      for (int j = 0; j < 2 && j < n && ok; ++j) {
+        const uint32_t ek = it_kv + 2 * j;
+        ok = kv_wait(ek) && kv_wait(ek + 1);
         if (!ok) break;
         tc_fence_after();
-        // prologue: S and dP of the first two tiles
-        for (int j = 0; j < 2 && j < n && ok; ++j) {
-          const uint32_t ek = it_kv + 2 * j;
-          ok = kv_wait(ek) && kv_wait(ek + 1);
-          if (!ok) break;
-          tc_fence_after();
-          int first, count;
-          tile_range(p, x, j, first, count);
-          issue_sd((G + j) & 1, ek, round16(count));
-          tc_commit(smem_u32(&bars->sd_full[(G + j) & 1]));
-          tc_commit(smem_u32(&bars->kv_empty[(ek + 1) % kStages]));   // V read by dP
-        }
-        // the previous item's dQ must have been read out before this item overwrites it
-        if (ok && item_cnt > 0) ok = mbar_wait(smem_u32(&bars->dq_empty), (item_cnt - 1) & 1, wc);
-        for (int j = 0; j < n && ok; ++j, ++G) {
-          const int b = G & 1;
-          ok = mbar_wait(smem_u32(&bars->ds_full[b]), (G >> 1) & 1, wc);
-          if (!ok) break;
-          tc_fence_after();
-          int first, count;
-          tile_range(p, x, j, first, count);
-          const int ksteps = round16(count) / 16;
-          const uint32_t ek = it_kv + 2 * j;
-          const uint64_t kb = kmn0 + (uint64_t)(((ek % kStages) * C::kSlotBytes) >> 4);
-          const uint32_t hi = tmem + 64 * b, lo = hi + 32;
-          for (int kk = 0; kk < ksteps; ++kk) {
-            const uint64_t bd = kb + (uint64_t)((kk * 16 * kRowBytes) >> 4);
-            tc_mma_ts(dq_tmem, hi + kk * 8, bd, idesc_dq, (j > 0 || kk > 0) ? 1u : 0u);
-            tc_mma_ts(dq_tmem, lo + kk * 8, bd, idesc_dq, 1u);
+        int first, count;
+        tile_range(p, x, j, first, count);
+        issue_sd((G + j) & 1, ek, round16(count));
+      }
+      // the previous item's dQ must have been read out before this item overwrites it
+      if (ok && item_cnt > 0) ok = mbar_wait_warp(smem_u32(&bars->dq_empty), (item_cnt - 1) & 1, wc);
+      for (int j = 0; j < n && ok; ++j, ++G) {
+        const int b = G & 1;
+        ok = mbar_wait_warp(smem_u32(&bars->ds_full[b]), (G >> 1) & 1, wc);
+        if (!ok) break;
+        tc_fence_after();
+        int first, count;
+        tile_range(p, x, j, first, count);
+        const int ksteps = round16(count) / 16;
+        const uint32_t ek = it_kv + 2 * j;
+        const uint64_t kb = kmn0 + (uint64_t)(((ek % kStages) * C::kSlotBytes) >> 4);
+        const uint32_t hi = tmem + 64 * b, lo = hi + 32;
+        if (elect_one()) {
+          if (ksteps == kNK / 16) {
+#pragma unroll
+            for (int kk = 0; kk < kNK / 16; ++kk) {
+              const uint64_t bd = kb + (uint64_t)((kk * 16 * kRowBytes) >> 4);
+              tc_mma_ts(dq_tmem, hi + kk * 8, bd, idesc_dq, (j > 0 || kk > 0) ? 1u : 0u);
+              tc_mma_ts(dq_tmem, lo + kk * 8, bd, idesc_dq, 1u);
+            }
+          } else {
+            for (int kk = 0; kk < ksteps; ++kk) {
+              const uint64_t bd = kb + (uint64_t)((kk * 16 * kRowBytes) >> 4);
+              tc_mma_ts(dq_tmem, hi + kk * 8, bd, idesc_dq, (j > 0 || kk > 0) ? 1u : 0u);
+              tc_mma_ts(dq_tmem, lo + kk * 8, bd, idesc_dq, 1u);
+            }
           }
           tc_commit(smem_u32(&bars->kv_empty[ek % kStages]));   // K read by S and dQ
-          if (j + 2 < n) {
-            // S and dP of tile j + 2 into buffer b, after dQ(j) has read dS(j) from it
-            const uint32_t e2 = it_kv + 2 * (j + 2);
-            ok = kv_wait(e2) && kv_wait(e2 + 1);
-            if (!ok) break;
-            tc_fence_after();
-            int f2, c2;
-            tile_range(p, x, j + 2, f2, c2);
-            issue_sd(b, e2, round16(c2));
-            tc_commit(smem_u32(&bars->sd_full[b]));
-            tc_commit(smem_u32(&bars->kv_empty[(e2 + 1) % kStages]));
-          }
         }
-        if (!ok) break;
-        it_kv += 2 * n;
+        __syncwarp();
+        if (j + 2 < n) {
+          // S and dP of tile j + 2 into buffer b, after dQ(j) has read dS(j) from it
+          const uint32_t e2 = it_kv + 2 * (j + 2);
+          ok = kv_wait(e2) && kv_wait(e2 + 1);
+          if (!ok) break;
+          tc_fence_after();
+          int f2, c2;
+          tile_range(p, x, j + 2, f2, c2);
+          issue_sd(b, e2, round16(c2));
+        }
+      }
+      if (!ok) break;
+      it_kv += 2 * n;
+      if (elect_one()) {
         tc_commit(smem_u32(&bars->dq_full));
         tc_commit(smem_u32(&bars->qo_empty));
       }
-      tc_commit(smem_u32(&bars->drain));
-      int dummy = 0;
-      WaitCtx dw{&dummy, nullptr, 2000000ull};
-      mbar_wait(smem_u32(&bars->drain), 0, dw);
+      __syncwarp();
     }
+    if (elect_one()) tc_commit(smem_u32(&bars->drain));
+    __syncwarp();
+    int dummy = 0;
+    WaitCtx dw{&dummy, nullptr, 2000000ull};
+    mbar_wait(smem_u32(&bars->drain), 0, dw);
     __syncwarp();
   } else if (warp == 2 || warp == 3) {
     // ========================================================= block reducer ==
