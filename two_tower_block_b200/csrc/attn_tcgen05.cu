@@ -164,6 +164,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int c = blockIdx.x;
   const int MT = p.R > 128 ? 2 : 1;
+  // a dependent combine launch may be scheduled now; it waits for this grid on the device
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   // ---------------------------------------------------------------- setup --
   {

@@ -355,16 +355,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           if (!has_s && !has_pv) return true;
           const uint32_t gs = G + t, gp = G + i;
           uint32_t ek = 0, ev = 0;
-          if (has_s) {
-            if (!s_buffer_free(gs)) return false;
-            ek = it + entry_k(t);
-            if (!ring_wait(ek)) return false;
-          }
+          // P(i) first: the warpgroup of tile i arrives on p_full once per tile, so this wait
+          // must not fall two of its arrivals behind (a parity wait cannot tell them apart);
+          // its next P needs S(i + 2), which the previous step issued just before this one
           if (has_pv) {
             if (!mbar_wait_cluster(bar(bars->p_full[gp & 1]), (gp >> 1) & 1, wc)) return false;
             ev = it + entry_v(i, n);
             if (!ring_wait(ev)) return false;
             if (i == 0 && !mbar_wait_cluster(bar(bars->o_empty), (seg_cnt & 1) ^ 1, wc)) return false;
+          }
+          if (has_s) {
+            if (!s_buffer_free(gs)) return false;
+            ek = it + entry_k(t);
+            if (!ring_wait(ek)) return false;
           }
           tc_fence_after();
           const int nk = has_s ? round16(tile_keys(p, x, sg.lo + t).count) : 0;

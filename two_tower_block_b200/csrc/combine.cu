@@ -13,6 +13,9 @@ constexpr int kThreads = 256;
 
 template <int D>
 __global__ void __launch_bounds__(kThreads) combine_kernel(const Problem p) {
+  // launched as a programmatic dependent of the attention kernel: wait until its grid has
+  // completed and its partials are visible
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int c = blockIdx.x;
   const SplitRecord rec = p.records[c];
   if (rec.unit < 0) return;
@@ -60,10 +63,19 @@ cudaError_t launch_exp2_selftest(const float* x, float* y, int n, cudaStream_t s
 }
 
 cudaError_t launch_combine(const Problem& p, cudaStream_t stream) {
-  dim3 grid(p.C, (p.R + kRowsPerBlock - 1) / kRowsPerBlock);
-  if (p.D == 128) combine_kernel<128><<<grid, kThreads, 0, stream>>>(p);
-  else combine_kernel<64><<<grid, kThreads, 0, stream>>>(p);
-  return cudaGetLastError();
+  // a programmatic dependent launch: the launch overlaps the attention kernel's tail and the
+  // kernel waits for the attention grid on the device
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.C, (p.R + kRowsPerBlock - 1) / kRowsPerBlock, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (p.D == 128) return cudaLaunchKernelEx(&cfg, combine_kernel<128>, p);
+  return cudaLaunchKernelEx(&cfg, combine_kernel<64>, p);
 }
 
 cudaError_t launch_wait_selftest(unsigned* err_word, unsigned long long limit_ns, cudaStream_t stream) {
