@@ -325,7 +325,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp == 1 && rank == 0 && have_work) {
     // ============================================= even CTA: 2-SM MMA issue ==
-    if (lane == 0) {
+    // The whole warp runs the control flow (waits and descriptors stay warp-uniform); one
+    // elected lane issues each burst of MMAs and its commits.
+    {
       uint32_t it = 0, q_it = 0, G = 0, seg_cnt = 0;
       bool ok = true;
       Unit x = ms->first;
@@ -336,18 +338,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const uint32_t idesc_s0 = idesc_bf16_f32(256, 0, 0, 0);
       const uint32_t idesc_pv = idesc_bf16_f32(256, kD, 0, 1);
       auto ring_wait = [&](uint32_t e) {
-        return mbar_wait_cluster(bar(bars->kv_ready[e % kStages]), (e / kStages) & 1, wc);
+        return mbar_wait_cluster_warp(bar(bars->kv_ready[e % kStages]), (e / kStages) & 1, wc);
       };
       // the S buffer of tile g was last used by tile g - 2: its softmax must have read it
       auto s_buffer_free = [&](uint32_t g) {
         if (g < 2) return true;
-        return mbar_wait_cluster(bar(bars->s_free[g & 1]), ((g >> 1) & 1) ^ 1, wc);
+        return mbar_wait_cluster_warp(bar(bars->s_free[g & 1]), ((g >> 1) & 1) ^ 1, wc);
       };
       for (; ok;) {
         const Segment sg = segment_of(x, start, end, c);
         const int n = sg.hi - sg.lo;
-        ok = mbar_wait_cluster(bar(bars->q_ready), q_it & 1, wc);
+        ok = mbar_wait_cluster_warp(bar(bars->q_ready), q_it & 1, wc);
         ++q_it;
+        if (!ok) break;
         // One step: S of tile t (when t < n) and P V of tile i (when 0 <= i), issued
         // interleaved.  Q is released after the segment's last S.
         auto step = [&](int t, int i) -> bool {
@@ -359,10 +362,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           // must not fall two of its arrivals behind (a parity wait cannot tell them apart);
           // its next P needs S(i + 2), which the previous step issued just before this one
           if (has_pv) {
-            if (!mbar_wait_cluster(bar(bars->p_full[gp & 1]), (gp >> 1) & 1, wc)) return false;
+            if (!mbar_wait_cluster_warp(bar(bars->p_full[gp & 1]), (gp >> 1) & 1, wc)) return false;
             ev = it + entry_v(i, n);
             if (!ring_wait(ev)) return false;
-            if (i == 0 && !mbar_wait_cluster(bar(bars->o_empty), (seg_cnt & 1) ^ 1, wc)) return false;
+            if (i == 0 && !mbar_wait_cluster_warp(bar(bars->o_empty), (seg_cnt & 1) ^ 1, wc)) return false;
           }
           if (has_s) {
             if (!s_buffer_free(gs)) return false;
@@ -378,24 +381,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           const uint64_t vd = add16(vdesc, (ev % kStages) * kEntryBytes);
           const uint32_t s_acc = tmem + 128 * (gs & 1), o_acc = tmem + 256 + 128 * (gp & 1);
           const uint32_t pv_acc0 = i >= 2 ? 1u : 0u;   // O_w starts at this warpgroup's first tile
+          if (elect_one()) {
 #pragma unroll
-          for (int kk = 0; kk < kD / 16; ++kk) {
-            if (has_s)
-              tc_mma2_ss(s_acc, add16(qdesc, (kk >> 2) * kHalf + (kk & 3) * 32),
-                         add16(kd, (kk >> 2) * (64 * kRowBytes) + (kk & 3) * 32), idesc_s, kk > 0);
-            if (kk < npv)
-              tc_mma2_ss(o_acc, add16(pd, (kk >> 2) * kHalf + (kk & 3) * 32), add16(vd, kk * 16 * kRowBytes),
-                         idesc_pv, kk > 0 ? 1u : pv_acc0);
+            for (int kk = 0; kk < kD / 16; ++kk) {
+              if (has_s)
+                tc_mma2_ss(s_acc, add16(qdesc, (kk >> 2) * kHalf + (kk & 3) * 32),
+                           add16(kd, (kk >> 2) * (64 * kRowBytes) + (kk & 3) * 32), idesc_s, kk > 0);
+              if (kk < npv)
+                tc_mma2_ss(o_acc, add16(pd, (kk >> 2) * kHalf + (kk & 3) * 32), add16(vd, kk * 16 * kRowBytes),
+                           idesc_pv, kk > 0 ? 1u : pv_acc0);
+            }
+            if (has_s) {
+              tc_commit2_both(bar(bars->s_full[gs & 1]));
+              tc_commit2_both(bar(bars->kv_empty[ek % kStages]));
+              if (t == n - 1) tc_commit2_both(bar(bars->q_empty));
+            }
+            if (has_pv) {
+              tc_commit2_both(bar(bars->pv_done[gp & 1][(gp >> 1) & 1]));
+              tc_commit2_both(bar(bars->kv_empty[ev % kStages]));
+            }
           }
-          if (has_s) {
-            tc_commit2_both(bar(bars->s_full[gs & 1]));
-            tc_commit2_both(bar(bars->kv_empty[ek % kStages]));
-            if (t == n - 1) tc_commit2_both(bar(bars->q_empty));
-          }
-          if (has_pv) {
-            tc_commit2_both(bar(bars->pv_done[gp & 1][(gp >> 1) & 1]));
-            tc_commit2_both(bar(bars->kv_empty[ev % kStages]));
-          }
+          __syncwarp();
           return true;
         };
         ok = step(0, -1);
@@ -403,7 +409,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         for (int j = 0; j < n && ok; ++j) ok = step(j + 2, j - 1);
         if (ok) ok = step(n, n - 1);
         if (!ok) break;
-        tc_commit2_both(bar(bars->o_full));
+        if (elect_one()) tc_commit2_both(bar(bars->o_full));
+        __syncwarp();
         it += 2 * n;
         G += n;
         ++seg_cnt;
@@ -573,11 +580,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   }
 
   // drain every 2-SM MMA before either CTA releases TMEM
-  if (warp == 1 && lane == 0) {
-    if (rank == 0) tc_commit2_both(bar(bars->drain));
+  if (warp == 1) {
+    // the lane that issued the MMAs commits (elect_one picks the same lane of a converged warp)
+    if (rank == 0 && elect_one()) tc_commit2_both(bar(bars->drain));
+    __syncwarp();
     int dummy = 0;
     WaitCtx dw{&dummy, nullptr, 2000000ull};
     mbar_wait(bar(bars->drain), 0, dw);
+    __syncwarp();
   }
   tc_fence_before();
   __syncthreads();

@@ -337,6 +337,11 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity,
     }
   }
 }
+// mbar_wait_cluster by every lane of a converged warp; the warp agrees on the result.
+__device__ __forceinline__ bool mbar_wait_cluster_warp(uint32_t bar, uint32_t parity, const WaitCtx& w) {
+  const bool ok = mbar_wait_cluster(bar, parity, w);
+  return __all_sync(0xffffffffu, ok);
+}
 __device__ __forceinline__ void tmem_alloc2(uint32_t dst_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem), "r"(ncols)
                : "memory");
