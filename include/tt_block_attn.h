@@ -296,10 +296,9 @@ TT_API tt_status_t tt_selftest_wait_timeout(int device, int timeout_us, tt_strea
 /* Numerics self test: evaluates on the device the library's FMA-pipe exp2 (range
  * reduction plus a fitted degree-3 polynomial, maximum relative error 7.5e-5 for
  * arguments in [-125, 127]) on the n host values x and writes the n results to y
- * (host).  The attention kernels do not use it: they call the hardware exp2
- * (ex2.approx), because offloading part of the softmax's exponentials to the FMA pipe
- * measured slower.  It stays a tested building block.  Synchronous; allocates its own
- * buffers. */
+ * (host).  The softmax of the default tcgen05 attention kernel computes one weight
+ * pair in eight with this routine and the rest with the hardware exp2 (ex2.approx).
+ * Synchronous; allocates its own buffers. */
 TT_API tt_status_t tt_selftest_exp2(int device, const float* x, float* y, int n);
 
 /* Host-only view of the work split (no GPU needed): for `num_units` units with

@@ -19,13 +19,11 @@ from two_tower_block_b200.workloads import WORKLOADS, bf16_bits, make_causal, ma
 pytestmark = pytest.mark.gpu
 
 # (kernel, plan-time tuning knobs): the tcgen05 kernel with two 64-key S buffers per
-# M-tile (default), with Q in TMEM and one 64-key buffer (TT_TCGEN05_VARIANT=1), with one
-# 128-key buffer (TT_TCGEN05_KEY_TILE=128), and the
+# M-tile (default), with one 128-key buffer (TT_TCGEN05_KEY_TILE=128), and the
 # transposed-PV kernel for head_dim 128 (TT_TCGEN05_VARIANT=2), the 2-SM kernel
 # (TT_TCGEN05_VARIANT=3; head_dim 128 with 128 % g == 0, else the default), the default kernel with
 # the split combine fused into its tail (TT_FUSED_COMBINE=1); the mma.sync baseline
 KERNELS = [pytest.param((ops.KERNEL_TCGEN05, {}), id="tcgen05"),
-           pytest.param((ops.KERNEL_TCGEN05, {"TT_TCGEN05_VARIANT": "1"}), id="tcgen05_qt"),
            pytest.param((ops.KERNEL_TCGEN05, {"TT_TCGEN05_KEY_TILE": "128"}), id="tcgen05_k128"),
            pytest.param((ops.KERNEL_TCGEN05, {"TT_TCGEN05_VARIANT": "2"}), id="tcgen05_pt"),
            pytest.param((ops.KERNEL_TCGEN05, {"TT_TCGEN05_VARIANT": "3"}), id="tcgen05_2sm"),

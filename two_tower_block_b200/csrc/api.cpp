@@ -293,8 +293,8 @@ tt_status_t tt_block_attn_plan(const tt_block_attn_desc* desc, int device, tt_pl
     // tiles, which they select unless a key tile is given
     if (const char* kv = std::getenv("TT_TCGEN05_VARIANT")) {
       const int v = std::atoi(kv);
-      P->variant = (v >= 1 && v <= 3) ? v : 0;
-      if (P->variant >= 2) P->key_tile = 128;
+      P->variant = (v == 2 || v == 3) ? v : 0;
+      if (P->variant != 0) P->key_tile = 128;
     }
     if (const char* kt = std::getenv("TT_TCGEN05_KEY_TILE")) {
       const int v = std::atoi(kt);
@@ -337,7 +337,7 @@ tt_status_t tt_block_attn_plan(const tt_block_attn_desc* desc, int device, tt_pl
   // the context lengths are equal, so no range carries a second segment (its extra Q load and
   // partial epilogue) at the cost of fewer than U idle SMs.  Ragged lengths are split as before.
   P->C_decode = P->C;
-  if (P->kernel == TT_KERNEL_TCGEN05 && P->variant <= 1 && d.num_ctas <= 0) {
+  if (P->kernel == TT_KERNEL_TCGEN05 && P->variant == 0 && d.num_ctas <= 0) {
     const long long U = (long long)d.batch * d.num_kv_heads;
     if (U > 0 && P->sm_count / U >= 2) P->C_decode = (int)(U * (P->sm_count / U));
   }
@@ -369,7 +369,7 @@ tt_status_t tt_block_attn_plan(const tt_block_attn_desc* desc, int device, tt_pl
   // separate combine kernel's launch.
   {
     const char* fc = std::getenv("TT_FUSED_COMBINE");
-    P->fused_combine = P->kernel == TT_KERNEL_TCGEN05 && P->variant <= 1 && P->C > 1 && P->C <= P->sm_count &&
+    P->fused_combine = P->kernel == TT_KERNEL_TCGEN05 && P->variant == 0 && P->C > 1 && P->C <= P->sm_count &&
                        fc && std::atoi(fc) == 1;
   }
   P->causal_pref = pref.empty() ? nullptr : reinterpret_cast<int*>(w + b_po + b_pl + b_rec + b_err);
@@ -475,7 +475,7 @@ tt_status_t tt_block_attn_paged(tt_plan_t plan, const void* q, const void* k_pag
   tt::Problem p = base_problem(plan);
   p.mode = tt::kDecode;
   p.NB = 1;
-  p.variant = plan->variant == 1 ? 1 : 0;  // the paged loads live in the default tcgen05 kernel (and the mma.sync one)
+  p.variant = 0;  // the paged loads live in the default tcgen05 kernel (and the mma.sync one)
   p.C = plan->variant == 3 ? plan->C_paged : plan->C_decode;
   p.ctx_stride = pages_per_seq * page_size;
   int shift = 0;

@@ -53,10 +53,10 @@ constexpr int kMaxRows = 256;
 constexpr int kRowBytes = 128;              // one 64-element bf16 row of a swizzled half
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
 
-template <int D, int NK, bool QT>
+template <int D, int NK>
 struct Cfg {
   static constexpr int kHalves = D / 64;
-  static constexpr int kBufs = QT ? 1 : 128 / NK;              // S buffers per M-tile
+  static constexpr int kBufs = 128 / NK;                       // S buffers per M-tile
   static constexpr int kSlotBytes = NK * kRowBytes * kHalves;  // one K or V tile
   static constexpr int kStages = (128 * 1024) / kSlotBytes;    // 128 KB ring
   static constexpr int kQBytes = kMaxRows * kRowBytes * kHalves;
@@ -77,8 +77,6 @@ struct Bars {
   uint64_t q_full, q_empty, tail, drain;
   uint64_t s_full[2][2], p_full[2][2];  // [M-tile][S buffer]
   uint64_t pv_done[2], o_full[2], o_empty[2];
-  uint64_t qt_full[2];                  // Q rows of M-tile m copied into TMEM (QT form)
-  uint64_t turn[2];                     // QT form with two M-tiles: softmax warpgroup m may start a tile
   uint64_t kv_full[16], kv_empty[16];
 };
 
@@ -146,11 +144,10 @@ __device__ __forceinline__ void fused_combine(const Problem& p, uint8_t* scratch
   }
 }
 
-template <int D, int NK, bool QT>
+template <int D, int NK>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tcgen05_kernel(const Problem p, const __grid_constant__ TmaMaps maps) {
-  using C = Cfg<D, NK, QT>;
-  static_assert(!QT || NK == 64, "the Q-in-TMEM form runs 64-key tiles");
+  using C = Cfg<D, NK>;
   constexpr int NBUF = C::kBufs;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -179,8 +176,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (tid == 0) {
     mbar_init(smem_u32(&bars->q_full), 1);
-    // one commit per M-tile issuer; in the QT form one arrival per softmax thread (its row copied)
-    mbar_init(smem_u32(&bars->q_empty), QT ? MT * 128 : MT);
+    mbar_init(smem_u32(&bars->q_empty), MT);  // one commit per M-tile issuer
     mbar_init(smem_u32(&bars->tail), 1);
     mbar_init(smem_u32(&bars->drain), MT);
     for (int m = 0; m < 2; ++m) {
@@ -189,8 +185,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(smem_u32(&bars->p_full[m][b]), 128);
       }
       mbar_init(smem_u32(&bars->pv_done[m]), 1);
-      mbar_init(smem_u32(&bars->qt_full[m]), 128);
-      mbar_init(smem_u32(&bars->turn[m]), 128);
       mbar_init(smem_u32(&bars->o_full[m]), 1);
       mbar_init(smem_u32(&bars->o_empty[m]), 128);
     }
@@ -352,8 +346,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint64_t vdesc0 = smem_desc_sw128(kv_s, NK * kRowBytes, 1024);
     const uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
     const uint32_t idesc_s0 = idesc_bf16_f32(128, 0, 0, 0);
-    const uint32_t s_tmem = tmem + m * (QT ? 64 : 128), o_tmem = tmem + 256 + m * D;
-    const uint32_t q_tmem = tmem + 128 + m * 64;   // QT form: Q_m as bf16 pairs, D / 2 columns
+    const uint32_t s_tmem = tmem + m * 128, o_tmem = tmem + 256 + m * D;
     // S = Q K^T of one tile into buffer `buf` (K in ring slot `slot`), then its commits
     auto issue_s = [&](int buf, uint32_t slot, int n_mma) {
       const uint32_t idesc = idesc_s0 | ((uint32_t)(n_mma >> 3) << 17);
@@ -363,10 +356,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * (kMaxRows * kRowBytes) + (kk & 3) * 32;
           const uint32_t koff = (kk >> 2) * (NK * kRowBytes) + (kk & 3) * 32;
-          if constexpr (QT)
-            tc_mma_ts(s_tmem + buf * NK, q_tmem + kk * 8, kd + (koff >> 4), idesc, kk > 0);
-          else
-            tc_mma_ss(s_tmem + buf * NK, qdesc + (off >> 4), kd + (koff >> 4), idesc, kk > 0);
+          tc_mma_ss(s_tmem + buf * NK, qdesc + (off >> 4), kd + (koff >> 4), idesc, kk > 0);
         }
         tc_commit(smem_u32(&bars->s_full[m][buf]));
         tc_commit(smem_u32(&bars->kv_empty[slot]));
@@ -380,8 +370,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (; ok;) {
       const Segment sg = segment_of(x, start, end, c);
       const int n = sg.hi - sg.lo;
-      if constexpr (QT) ok = mbar_wait_warp(smem_u32(&bars->qt_full[m]), seg_cnt & 1, wc);
-      else ok = mbar_wait_warp(smem_u32(&bars->q_full), q_it & 1, wc);
+      ok = mbar_wait_warp(smem_u32(&bars->q_full), q_it & 1, wc);
       ++q_it;
       if (!ok) break;
       tc_fence_after();
@@ -430,7 +419,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tb += n;
       if (elect_one()) {
         tc_commit(smem_u32(&bars->o_full[m]));
-        if constexpr (!QT) tc_commit(smem_u32(&bars->q_empty));
+        tc_commit(smem_u32(&bars->q_empty));
       }
       __syncwarp();
       ++seg_cnt;
@@ -453,40 +442,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r = m * 128 + row;         // packed row of the unit
     if (m < MT) {
       const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
-      const uint32_t s_base = tmem + lane_off + m * (QT ? 64 : 128);  // + buffer * NK
+      const uint32_t s_base = tmem + lane_off + m * 128;  // + buffer * NK
       const uint32_t o_addr = tmem + lane_off + 256 + m * D;
       float* stage = epi + (warp - 4) * 32 * 32;
-      uint32_t G = 0, seg_cnt = 0, q_it = 0;
+      uint32_t G = 0, seg_cnt = 0;
       bool ok = true;
       Unit x = sh->first;
-      // QT form: this thread's Q row (row r of the 128-byte-swizzled shared tile) into TMEM lane
-      // `row` of Q_m, then the shared tile is released.  Called once the M-tile's S MMAs of the
-      // previous segment have all completed (its last S was consumed), so Q_m is free.
-      auto copy_q = [&]() -> bool {
-        if (!mbar_wait(smem_u32(&bars->q_full), q_it & 1, wc)) return false;
-        ++q_it;
-        const uint32_t q_addr = tmem + lane_off + 128 + m * 64;
-#pragma unroll
-        for (int hf = 0; hf < C::kHalves; ++hf) {
-          uint32_t v[32];
-#pragma unroll
-          for (int cq = 0; cq < 8; ++cq) {
-            const uint4 u = *reinterpret_cast<const uint4*>(smem + hf * (kMaxRows * kRowBytes) + r * kRowBytes +
-                                                            ((cq ^ (r & 7)) << 4));
-            v[4 * cq] = u.x;
-            v[4 * cq + 1] = u.y;
-            v[4 * cq + 2] = u.z;
-            v[4 * cq + 3] = u.w;
-          }
-          tmem_st32(q_addr + 32 * hf, v);
-        }
-        tc_wait_st();
-        tc_fence_before();
-        mbar_arrive(smem_u32(&bars->qt_full[m]));
-        mbar_arrive(smem_u32(&bars->q_empty));
-        return true;
-      };
-      if constexpr (QT) ok = copy_q();
       for (; ok;) {
         const Segment sg = segment_of(x, start, end, c);
         float m_ref = -INFINITY, l = 0.f;
@@ -534,12 +495,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int b = G % NBUF;
           const uint32_t s_addr = s_base + b * NK;
           ok = mbar_wait(smem_u32(&bars->s_full[m][b]), (G / NBUF) & 1, wc);
-          // QT form, two M-tiles: the warpgroups take turns tile by tile (M-tile 0 first), so one
-          // softmax runs while the other M-tile's P V and next S occupy the tensor core
-          if constexpr (QT) {
-            if (ok && MT == 2 && (m == 1 || G > 0))
-              ok = mbar_wait(smem_u32(&bars->turn[m]), (m == 1 ? G : G - 1) & 1, wc);
-          }
           if (!ok) break;
           tc_fence_after();
           // (128-key tiles keep a single masked path: a second copy of their 128-register body
@@ -550,19 +505,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = count == NK ? tile(std::true_type{}, count, s_addr, i == sg.lo)
                              : tile(std::false_type{}, count, s_addr, i == sg.lo);
           if (!ok) break;
-          if constexpr (QT) {
-            if (MT == 2) mbar_arrive(smem_u32(&bars->turn[m ^ 1]));
-          }
           tc_wait_st();
           tc_fence_before();
           mbar_arrive(smem_u32(&bars->p_full[m][b]));
         }
         if (!ok) break;
-        // QT form: the next segment's Q goes into TMEM before this epilogue, so its first S
-        // MMAs overlap the epilogue
-        if constexpr (QT) {
-          if (!sg.last && !copy_q()) break;
-        }
         // ---- epilogue: O / l to the output (or the segment's partial) ----
         ok = mbar_wait(smem_u32(&bars->o_full[m]), seg_cnt & 1, wc);
         if (!ok) break;
@@ -634,30 +581,30 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (p.grid_bar != nullptr) fused_combine<D>(p, smem + C::kEpiOff, *(volatile int*)&sh->abort_flag != 0);
 }
 
-template <int D, int NK, bool QT>
+template <int D, int NK>
 void set_smem_attr() {
-  cudaFuncSetAttribute(attn_tcgen05_kernel<D, NK, QT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                       Cfg<D, NK, QT>::kSmemBytes);
+  cudaFuncSetAttribute(attn_tcgen05_kernel<D, NK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       Cfg<D, NK>::kSmemBytes);
 }
 
-template <int D, int NK, bool QT = false>
+template <int D, int NK>
 cudaError_t launch(const Problem& p, const TmaMaps& maps, cudaStream_t stream) {
   if (p.grid_bar == nullptr) {
-    attn_tcgen05_kernel<D, NK, QT><<<p.C, kThreads, Cfg<D, NK, QT>::kSmemBytes, stream>>>(p, maps);
+    attn_tcgen05_kernel<D, NK><<<p.C, kThreads, Cfg<D, NK>::kSmemBytes, stream>>>(p, maps);
     return cudaGetLastError();
   }
   // cooperative: every CTA must be resident at once for the grid barrier of the fused combine
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.C, 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = Cfg<D, NK, QT>::kSmemBytes;
+  cfg.dynamicSmemBytes = Cfg<D, NK>::kSmemBytes;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeCooperative;
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, attn_tcgen05_kernel<D, NK, QT>, p, maps);
+  return cudaLaunchKernelEx(&cfg, attn_tcgen05_kernel<D, NK>, p, maps);
 }
 
 }  // namespace
@@ -666,21 +613,16 @@ bool tcgen05_key_tile_supported(int key_tile) { return key_tile == 64 || key_til
 
 cudaError_t launch_attn_tcgen05(const Problem& p, const TmaMaps& maps, cudaStream_t stream) {
   static const bool attr_done = [] {
-    set_smem_attr<128, 128, false>();
-    set_smem_attr<128, 64, false>();
-    set_smem_attr<64, 128, false>();
-    set_smem_attr<64, 64, false>();
-    set_smem_attr<128, 64, true>();
-    set_smem_attr<64, 64, true>();
+    set_smem_attr<128, 128>();
+    set_smem_attr<128, 64>();
+    set_smem_attr<64, 128>();
+    set_smem_attr<64, 64>();
     return true;
   }();
   (void)attr_done;
   if (!tcgen05_key_tile_supported(p.key_tile)) return cudaErrorInvalidValue;
   // variant 2: head_dim 128 with 128-key tiles on the transposed-PV kernel (attn_tcgen05_pt.cu)
   if (p.D == 128 && p.key_tile == 128 && p.variant == 2) return launch_attn_pt(p, maps, stream);
-  // variant 1: 64-key tiles with Q in TMEM (the S MMAs read only K from shared memory)
-  if (p.variant == 1 && p.key_tile == 64)
-    return p.D == 128 ? launch<128, 64, true>(p, maps, stream) : launch<64, 64, true>(p, maps, stream);
   if (p.D == 128) return p.key_tile == 128 ? launch<128, 128>(p, maps, stream) : launch<128, 64>(p, maps, stream);
   return p.key_tile == 128 ? launch<64, 128>(p, maps, stream) : launch<64, 64>(p, maps, stream);
 }

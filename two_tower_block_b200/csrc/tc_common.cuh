@@ -51,6 +51,10 @@ __device__ __forceinline__ float tile_row_max(const uint32_t* v, int count) {
 // (round_pair_bf16) and written to TMEM as pairs over the first columns of the S buffer: keys
 // [32ch, 32ch+32) -> columns [16ch, 16ch+16).  Returns the row sum of the
 // rounded weights, so that numerator and denominator use the same values.
+// One pair in kPolyEvery is computed on the FMA pipe (exp2_poly2, relative error 7.5e-5,
+// far below the bf16 rounding that follows) instead of the MUFU, whose exp2 throughput
+// bounds this loop; one in eight measured fastest (one in four or three was slower).
+constexpr int kPolyEvery = 8;
 template <int NK, bool kFull>
 __device__ __forceinline__ float tile_exp_store(const uint32_t* v, int count, float c, float m_ref,
                                                 uint32_t s_addr) {
@@ -65,7 +69,15 @@ __device__ __forceinline__ float tile_exp_store(const uint32_t* v, int count, fl
     for (int k = 0; k < 16; ++k) {
       const int c0 = 32 * ch + 2 * k;
       const float2 x = __ffma2_rn(make_float2(__uint_as_float(v[c0]), __uint_as_float(v[c0 + 1])), c2, nm2);
-      float a = fast_exp2(x.x), b = fast_exp2(x.y);
+      float a, b;
+      if (k % kPolyEvery == kPolyEvery - 1) {
+        const float2 e = exp2_poly2(x);
+        a = e.x;
+        b = e.y;
+      } else {
+        a = fast_exp2(x.x);
+        b = fast_exp2(x.y);
+      }
       if (!kFull) {
         a = c0 < count ? a : 0.f;
         b = c0 + 1 < count ? b : 0.f;
