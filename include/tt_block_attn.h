@@ -297,7 +297,8 @@ TT_API tt_status_t tt_selftest_wait_timeout(int device, int timeout_us, tt_strea
  * reduction plus a fitted degree-3 polynomial, maximum relative error 7.5e-5 for
  * arguments in [-125, 127]) on the n host values x and writes the n results to y
  * (host).  The softmax of the default tcgen05 attention kernel computes one weight
- * pair in eight with this routine and the rest with the hardware exp2 (ex2.approx).
+ * pair in eight with this routine, the unmasking scan one pair in four, and the rest
+ * with the hardware exp2 (ex2.approx).
  * Synchronous; allocates its own buffers. */
 TT_API tt_status_t tt_selftest_exp2(int device, const float* x, float* y, int n);
 

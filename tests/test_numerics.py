@@ -3,7 +3,8 @@
 The routine computes 2^x without the MUFU: x = j + f, j = round(x) via the
 1.5 * 2^23 shifter, |f| <= 1/2, 2^f by a degree-3 polynomial, 2^j added to the
 exponent field.  The softmax of the default tcgen05 kernel computes one weight pair
-in eight with it (the rest with the hardware ex2.approx).  The CPU test re-derives the
+in eight with it and the unmasking scan one pair in four (the rest with the hardware
+ex2.approx).  The CPU test re-derives the
 error bound of the recipe with the coefficients the library uses (read from its
 source) in float32 numpy; the GPU test checks the device routine against float64
 exp2 through the self-test entry point."""

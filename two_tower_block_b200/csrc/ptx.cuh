@@ -74,7 +74,8 @@ __device__ __forceinline__ float fast_exp2(float x) {
 // 2^x for a pair of arguments on the FMA and integer pipes (no MUFU), for x in
 // [-125, 127]; arguments below -125 are clamped there (2^-125 ~ 2.4e-38).  The softmax of
 // the default tcgen05 kernel computes one weight pair in eight with it (tc_common.cuh:
-// tile_exp_store); the numerics self test evaluates it on its own.
+// tile_exp_store) and the unmasking scan one pair in four (unmask.cu); the numerics self test
+// evaluates it on its own.
 // Range reduction x = j + f with j = round(x) taken by the 1.5 * 2^23 shifter and
 // |f| <= 1/2; 2^f by a degree-3 polynomial whose coefficients were fitted for
 // this library by iteratively reweighted least squares on the relative error

@@ -13,7 +13,8 @@
 // 2^(x - max), argmax) per thread in the log2 domain, merged across the CTA; the
 // probability of the argmax token is 1 / sum.  Each thread takes its logits in batches
 // of 32 (four 16-byte loads in flight), rescaling its sum once per batch; 1024 threads
-// per row keep 64 KB of loads in flight per SM.  Kernel 2 is launched as a
+// per row keep 64 KB of loads in flight per SM.  One exponential pair in four is computed
+// on the FMA pipe (ptx.cuh: exp2_poly2) to relieve the MUFU.  Kernel 2 is launched as a
 // programmatic dependent of kernel 1, so its launch overlaps the scan.  Kernel 2: one CTA per sequence
 // applies the commit rule to tokens and mask.
 #include "unmask.h"
@@ -130,7 +131,9 @@ __global__ void __launch_bounds__(kScanThreads, 1)
         for (int k = 0; k < 4; ++k) {
           const float2 t = __ffma2_rn(make_float2(__uint_as_float(w[k] << 16), __uint_as_float(w[k] & 0xFFFF0000u)),
                                       c2, nm2);
-          const float2 e = make_float2(fast_exp2(t.x), fast_exp2(t.y));
+          // one pair in four on the FMA pipe (exp2_poly2, relative error 7.5e-5): the MUFU's
+          // exp2 rate bounds the scan together with its loads
+          const float2 e = k == 3 ? exp2_poly2(t) : make_float2(fast_exp2(t.x), fast_exp2(t.y));
           if (k & 1) s1 = __fadd2_rn(s1, e);
           else s0 = __fadd2_rn(s0, e);
         }
