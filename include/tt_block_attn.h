@@ -104,7 +104,8 @@ typedef struct {
   size_t workspace_bytes;  /* device scratch owned by the plan                        */
   int sm_count;
   int variant;             /* tcgen05 kernel form: 0 default, 2 transposed PV, 3 2-SM pairs */
-  int fused_combine;       /* non-zero: the split combine runs in the attention kernel's tail */
+  int fused_combine;       /* non-zero: decode calls run the split combine in the attention
+                              kernel's tail (one launch per call)                          */
 } tt_plan_info;
 
 /* Create a plan: validates the descriptor, picks the kernel and the work split

@@ -97,8 +97,13 @@ struct tt_plan_s {
   float* part_lse = nullptr;
   tt::SplitRecord* records = nullptr;
   unsigned* err_word = nullptr;
-  unsigned long long* grid_bar = nullptr;  // fused combine's grid barrier (in the error-word block)
-  bool fused_combine = false;
+  // fused combine: per-range arrival counts (only growing) of the decode and paged calls
+  // (C_decode ranges) and of the block-causal calls (C ranges); each launch kind keeps its own
+  // so that every range of a launch has seen the same number of launches
+  unsigned* arr_decode = nullptr;
+  unsigned* arr_causal = nullptr;
+  bool fused_combine = false;   // block-causal calls combine in the attention kernel's tail
+  bool fused_decode = false;    // decode and paged calls do
   int* causal_pref = nullptr;
   long long causal_T = 0;
   int causal_NB = 0;
@@ -129,13 +134,17 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 void prof_mark(tt_plan_t plan, int kid, cudaStream_t s, bool begin) {
   if (!plan->prof_on) return;
+  if (plan->prof_n >= kProfMax) return;
+  // in a stream being captured into a graph, the record must become a graph node of its own
+  // (cudaEventRecordExternal) for its timestamp to be readable after the graph has run
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  cudaStreamIsCapturing(s, &cs);
+  const unsigned flags = cs == cudaStreamCaptureStatusActive ? cudaEventRecordExternal : cudaEventRecordDefault;
   if (begin) {
-    if (plan->prof_n >= kProfMax) return;
-    cudaEventRecord(plan->prof_ev[2 * plan->prof_n], s);
+    cudaEventRecordWithFlags(plan->prof_ev[2 * plan->prof_n], s, flags);
     plan->prof_kid[plan->prof_n] = kid;
   } else {
-    if (plan->prof_n >= kProfMax) return;
-    cudaEventRecord(plan->prof_ev[2 * plan->prof_n + 1], s);
+    cudaEventRecordWithFlags(plan->prof_ev[2 * plan->prof_n + 1], s, flags);
     plan->prof_n++;
   }
 }
@@ -160,7 +169,7 @@ tt::Problem base_problem(tt_plan_t plan) {
   p.err_word = plan->err_word;
   p.wait_limit_ns = (unsigned long long)(d.wait_timeout_us > 0 ? d.wait_timeout_us : 1000000) * 1000ull;
   p.variant = plan->variant;
-  p.grid_bar = plan->fused_combine ? plan->grid_bar : nullptr;
+  p.arrivals = nullptr;
   return p;
 }
 
@@ -220,7 +229,7 @@ tt_status_t launch_all(tt_plan_t plan, const tt::Problem& p, cudaStream_t s) {
   }
   prof_mark(plan, 0, s, false);
   if (e != cudaSuccess) return cuda_fail(e, "attention kernel launch");
-  if (p.C > 1 && p.grid_bar == nullptr) {
+  if (p.C > 1 && p.arrivals == nullptr) {
     prof_mark(plan, 1, s, true);
     e = tt::launch_combine(p, s);
     prof_mark(plan, 1, s, false);
@@ -337,9 +346,13 @@ tt_status_t tt_block_attn_plan(const tt_block_attn_desc* desc, int device, tt_pl
   // the context lengths are equal, so no range carries a second segment (its extra Q load and
   // partial epilogue) at the cost of fewer than U idle SMs.  Ragged lengths are split as before.
   P->C_decode = P->C;
+  bool decode_aligned = false;   // every unit of a decode call gets at least two ranges
   if (P->kernel == TT_KERNEL_TCGEN05 && P->variant == 0 && d.num_ctas <= 0) {
     const long long U = (long long)d.batch * d.num_kv_heads;
-    if (U > 0 && P->sm_count / U >= 2) P->C_decode = (int)(U * (P->sm_count / U));
+    if (U > 0 && P->sm_count / U >= 2) {
+      P->C_decode = (int)(U * (P->sm_count / U));
+      decode_aligned = true;
+    }
   }
   // scratch layout (256-byte aligned pieces).  A 2-SM plan runs one range per SM pair, but
   // its paged calls run on the one-CTA-per-SM kernel: room for one range per SM as well.
@@ -351,7 +364,8 @@ tt_status_t tt_block_attn_plan(const tt_block_attn_desc* desc, int device, tt_pl
   const size_t b_rec = up((size_t)Cmax * sizeof(tt::SplitRecord));
   const size_t b_err = 256;
   const size_t b_pref = up(pref.size() * sizeof(int));
-  P->ws_bytes = b_po + b_pl + b_rec + b_err + b_pref;
+  const size_t b_arr = up((size_t)2 * Cmax * sizeof(unsigned));
+  P->ws_bytes = b_po + b_pl + b_rec + b_err + b_pref + b_arr;
   e = cudaMalloc(&P->ws, P->ws_bytes);
   if (e != cudaSuccess) {
     delete P;
@@ -362,18 +376,31 @@ tt_status_t tt_block_attn_plan(const tt_block_attn_desc* desc, int device, tt_pl
   P->part_lse = reinterpret_cast<float*>(w + b_po);
   P->records = reinterpret_cast<tt::SplitRecord*>(w + b_po + b_pl);
   P->err_word = reinterpret_cast<unsigned*>(w + b_po + b_pl + b_rec);
-  P->grid_bar = reinterpret_cast<unsigned long long*>(w + b_po + b_pl + b_rec + 128);
-  // TT_FUSED_COMBINE=1: the default tcgen05 kernel combines the cut units itself when all
-  // its CTAs can be resident at once (one per SM): a cooperative launch with a grid
-  // barrier at the end.  Off by default: waiting for the slowest CTA costs more than the
-  // separate combine kernel's launch.
+  P->arr_decode = reinterpret_cast<unsigned*>(w + b_po + b_pl + b_rec + b_err + b_pref);
+  P->arr_causal = P->arr_decode + Cmax;
+  // The fused combine: the default tcgen05 kernel combines the cut units itself, in a
+  // cooperative launch (all CTAs resident, one per SM) in which the ranges of each cut unit
+  // wait for one another and share its rows, so a call is one launch.  It is the default for
+  // decode and paged calls when every unit gets at least two ranges (the aligned split above)
+  // and a range holds at most 32 key tiles at the plan's context capacity: there the
+  // combine's fixed cost is a large share of a short step (L = 4096: step 36.0 -> 33.3 us).
+  // With long ranges the step gains little (L = 131072: 154.9 -> 153.5 us) while the
+  // attention kernel's own time grows by the combine's work; with fewer ranges per unit
+  // (ragged batches: 213 vs 225 us at B = 64) and for block-causal calls the separate combine
+  // kernel measured faster.  TT_FUSED_COMBINE=1 fuses every call of the plan, =0 none.
   {
     const char* fc = std::getenv("TT_FUSED_COMBINE");
-    P->fused_combine = P->kernel == TT_KERNEL_TCGEN05 && P->variant == 0 && P->C > 1 && P->C <= P->sm_count &&
-                       fc && std::atoi(fc) == 1;
+    const int force = fc ? std::atoi(fc) : -1;
+    const bool can = P->kernel == TT_KERNEL_TCGEN05 && P->variant == 0 && P->C > 1 && P->C <= P->sm_count;
+    P->fused_combine = can && force == 1;
+    const long long unit_tiles = 1 + (long long)tt::ceil_div(d.ctx_capacity, P->key_tile);
+    const bool short_ranges =
+        decode_aligned && unit_tiles * d.batch * d.num_kv_heads <= 32LL * std::max(P->C_decode, 1);
+    P->fused_decode = can && P->C_decode <= P->sm_count && (force == 1 || (force != 0 && short_ranges));
   }
   P->causal_pref = pref.empty() ? nullptr : reinterpret_cast<int*>(w + b_po + b_pl + b_rec + b_err);
   e = cudaMemset(P->err_word, 0, b_err);
+  if (e == cudaSuccess) e = cudaMemset(P->arr_decode, 0, b_arr);
   if (e == cudaSuccess && !pref.empty())
     e = cudaMemcpy(P->causal_pref, pref.data(), pref.size() * sizeof(int), cudaMemcpyHostToDevice);
   if (e != cudaSuccess) {
@@ -420,7 +447,7 @@ tt_status_t tt_block_attn_plan_get_info(tt_plan_t plan, tt_plan_info* info) {
   info->workspace_bytes = plan->ws_bytes;
   info->sm_count = plan->sm_count;
   info->variant = plan->kernel == TT_KERNEL_TCGEN05 ? plan->variant : 0;
-  info->fused_combine = plan->fused_combine ? 1 : 0;
+  info->fused_combine = plan->fused_decode ? 1 : 0;
   return TT_OK;
 }
 
@@ -437,6 +464,7 @@ tt_status_t tt_block_attn(tt_plan_t plan, const void* q, const void* k_ctx, cons
   DeviceGuard guard(plan->device);
   tt::Problem p = base_problem(plan);
   p.C = plan->C_decode;
+  p.arrivals = plan->fused_decode ? plan->arr_decode : nullptr;
   p.mode = tt::kDecode;
   p.NB = 1;
   p.ctx_stride = d.ctx_capacity;
@@ -477,6 +505,7 @@ tt_status_t tt_block_attn_paged(tt_plan_t plan, const void* q, const void* k_pag
   p.NB = 1;
   p.variant = 0;  // the paged loads live in the default tcgen05 kernel (and the mma.sync one)
   p.C = plan->variant == 3 ? plan->C_paged : plan->C_decode;
+  p.arrivals = plan->fused_decode ? plan->arr_decode : nullptr;
   p.ctx_stride = pages_per_seq * page_size;
   int shift = 0;
   while ((1 << shift) < page_size) ++shift;
@@ -510,6 +539,7 @@ tt_status_t tt_block_attn_block_causal(tt_plan_t plan, const void* q, const void
   tt::Problem p = base_problem(plan);
   p.mode = tt::kBlockCausal;
   p.NB = plan->causal_NB;
+  p.arrivals = plan->fused_combine ? plan->arr_causal : nullptr;
   p.ctx_stride = d.seq_len;
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.k_ctx = static_cast<const __nv_bfloat16*>(k_ctx);

@@ -88,59 +88,60 @@ struct Shared {
 };
 static_assert(sizeof(Bars) + sizeof(Shared) <= 512, "barrier block overflows its shared-memory slot");
 
-// Fused split combine (cooperative launch only): every CTA arrives at a grid barrier once
-// its segments and its split record are written, then the CTAs share the rows of the cut
-// units, one warp per row.  `scratch` holds C records and C indices.  The wait is bounded;
-// a CTA that gave up (or whose pipeline aborted) combines nothing and the error word says so.
+// Fused split combine (cooperative launch only: every CTA is resident).  Once its segments and
+// partials are written, each CTA adds one to its range's arrival count; every range does so
+// exactly once per launch, so all counts of a launch are equal.  For each cut unit with a
+// segment in this range (at most two: the unit holding the range's first tile and the one
+// holding its last), the CTA waits until every range of that unit has reached its own count,
+// then combines its share of the unit's rows: rows [i R / n, (i + 1) R / n) for the i-th of the
+// unit's n ranges, one warp per row.  No CTA waits for ranges outside its units.  The waits
+// are bounded; a CTA that gave up (or whose pipeline aborted) combines nothing and the error
+// word says so.
 template <int D>
-__device__ __forceinline__ void fused_combine(const Problem& p, uint8_t* scratch, bool aborted) {
-  __shared__ int s_go, s_ncut;
+__device__ __forceinline__ void fused_combine(const Problem& p, long long T, long long start, long long end,
+                                              const Unit& first, bool aborted) {
+  __shared__ unsigned s_k;
+  __shared__ int s_ok;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int c = blockIdx.x;
   __syncthreads();  // every write of this CTA precedes its arrival
   if (tid == 0) {
     __threadfence();
-    const unsigned long long old = atomicAdd(p.grid_bar, 1ull);
-    const unsigned long long target = (old / (unsigned long long)p.C + 1ull) * (unsigned long long)p.C;
-    const unsigned long long t0 = globaltimer_ns();
-    bool ok = true;
-    while (ld_acquire_gpu(p.grid_bar) < target) {
-      if (globaltimer_ns() - t0 > p.wait_limit_ns) {
-        raise_error(p.err_word, kErrTimeout);
-        ok = false;
-        break;
+    s_k = atomicAdd(p.arrivals + c, 1u) + 1u;
+  }
+  __syncthreads();
+  if (start >= end || aborted) return;
+  const unsigned k = s_k;
+  const int Ce = used_ranges(T, p.C);
+  Unit last = first;
+  while (last.Tu + last.tiles < end) last = make_unit(p, last.u + 1, last.Tu + last.tiles);
+  for (int which = 0; which < 2; ++which) {
+    const Unit x = which == 0 ? first : last;
+    if (which == 1 && last.u == first.u) break;
+    if (x.Tu >= start && x.Tu + x.tiles <= end) continue;  // whole in this range: not cut
+    const int c0 = range_of_tile(T, Ce, x.Tu), c1 = range_of_tile(T, Ce, x.Tu + x.tiles - 1);
+    if (warp == 0) {
+      bool ok = true;
+      const unsigned long long t0 = globaltimer_ns();
+      for (int cc = c0 + lane; cc <= c1 && ok; cc += 32) {
+        while (ld_acquire_gpu_u32(p.arrivals + cc) < k) {
+          if (globaltimer_ns() - t0 > p.wait_limit_ns) {
+            raise_error(p.err_word, kErrTimeout);
+            ok = false;
+            break;
+          }
+          __nanosleep(32);
+        }
       }
-      __nanosleep(64);
+      ok = __all_sync(0xffffffffu, ok);
+      if (lane == 0) s_ok = ok;
     }
-    __threadfence();
-    s_go = ok && !aborted;
-  }
-  __syncthreads();
-  if (!s_go) return;
-  SplitRecord* recs = reinterpret_cast<SplitRecord*>(scratch);
-  int* cut = reinterpret_cast<int*>(scratch + p.C * sizeof(SplitRecord));
-  for (int i = tid; i < p.C; i += kThreads) {
-    const int4 v = __ldcg(reinterpret_cast<const int4*>(p.records + i));
-    recs[i] = SplitRecord{v.x, v.y, v.z, v.w};
-  }
-  __syncthreads();
-  if (warp == 0) {
-    int n = 0;
-    for (int base = 0; base < p.C; base += 32) {
-      const int i = base + lane;
-      const bool is_cut = i < p.C && recs[i].unit >= 0;
-      const unsigned m = __ballot_sync(0xffffffffu, is_cut);
-      if (is_cut) cut[n + __popc(m & ((1u << lane) - 1u))] = i;
-      n += __popc(m);
-    }
-    if (lane == 0) s_ncut = n;
-  }
-  __syncthreads();
-  const int nw = kThreads / 32;
-  const long long jobs = (long long)s_ncut * p.R;
-  for (long long job = (long long)blockIdx.x * nw + warp; job < jobs; job += (long long)p.C * nw) {
-    const int k = (int)(job / p.R), r = (int)(job - (long long)k * p.R);
-    const int c = cut[k];
-    combine_row<D>(p, c, recs[c], r, lane);
+    __syncthreads();
+    if (!s_ok) return;
+    const int n = c1 - c0 + 1, i = c - c0;
+    const SplitRecord rec{x.u, c1, x.Tu == range_start(T, Ce, c0) ? 0 : 1, 0};
+    const int r0 = (int)((long long)i * p.R / n), r1 = (int)((long long)(i + 1) * p.R / n);
+    for (int r = r0 + warp; r < r1; r += kThreads / 32) combine_row<D>(p, c0, rec, r, lane);
   }
 }
 
@@ -578,7 +579,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem, 512);
-  if (p.grid_bar != nullptr) fused_combine<D>(p, smem + C::kEpiOff, *(volatile int*)&sh->abort_flag != 0);
+  if (p.arrivals != nullptr)
+    fused_combine<D>(p, T, start, end, sh->first, *(volatile int*)&sh->abort_flag != 0);
 }
 
 template <int D, int NK>
@@ -589,11 +591,11 @@ void set_smem_attr() {
 
 template <int D, int NK>
 cudaError_t launch(const Problem& p, const TmaMaps& maps, cudaStream_t stream) {
-  if (p.grid_bar == nullptr) {
+  if (p.arrivals == nullptr) {
     attn_tcgen05_kernel<D, NK><<<p.C, kThreads, Cfg<D, NK>::kSmemBytes, stream>>>(p, maps);
     return cudaGetLastError();
   }
-  // cooperative: every CTA must be resident at once for the grid barrier of the fused combine
+  // cooperative: every CTA must be resident at once for the waits of the fused combine
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.C, 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);

@@ -49,10 +49,11 @@ struct Problem {
   unsigned long long wait_limit_ns;
   int variant;          // tcgen05 kernel: 0 = S/P aliasing in TMEM (default), 2 = transposed PV,
                         // 3 = 2-SM pairs (head_dim 128)
-  // default tcgen05 kernel launched cooperatively: the CTAs meet at this grid barrier
-  // (a counter that only grows) and combine the cut units themselves; null: the
-  // separate combine kernel runs instead
-  unsigned long long* grid_bar;
+  // default tcgen05 kernel launched cooperatively: every CTA adds one to its range's entry
+  // (per-range launch counts that only grow) once its partials are written, waits for the
+  // ranges that share its cut units to reach the same count, and combines its share of
+  // those units' rows; null: the separate combine kernel runs instead
+  unsigned* arrivals;
   // paged context cache (decode only; null page_table: contiguous k_ctx / v_ctx).
   // k_ctx / v_ctx then point at pools [num_pages][Hkv][page_size][D]; context position
   // pos of sequence n sits in page page_table[n * pages_per_seq + (pos >> page_shift)]
