@@ -141,7 +141,7 @@ __device__ __forceinline__ void fused_combine(const Problem& p, long long T, lon
     const int n = c1 - c0 + 1, i = c - c0;
     const SplitRecord rec{x.u, c1, x.Tu == range_start(T, Ce, c0) ? 0 : 1, 0};
     const int r0 = (int)((long long)i * p.R / n), r1 = (int)((long long)(i + 1) * p.R / n);
-    for (int r = r0 + warp; r < r1; r += kThreads / 32) combine_row<D>(p, c0, rec, r, lane);
+    for (int r = r0 + warp; r < r1; r += kThreads / 32) combine_row<D, 16>(p, c0, rec, r, lane);
   }
 }
 

@@ -14,9 +14,10 @@
 
 namespace tt {
 
-template <int D>
+// kGroup rows are loaded per round: 8 in the separate kernel (more would cost occupancy), 16 in
+// the attention kernel's tail, whose registers are there anyway.
+template <int D, int kGroup = 8>
 __device__ __forceinline__ void combine_row(const Problem& p, int c, const SplitRecord& rec, int r, int lane) {
-  constexpr int kGroup = 8;
   constexpr int V = D / 32;  // columns per lane
   const Unit x = make_unit(p, rec.unit, 0);
   const int nseg = rec.last_range - c + 1;
