@@ -382,7 +382,7 @@ tt_status_t tt_block_attn_plan(const tt_block_attn_desc* desc, int device, tt_pl
   // cooperative launch (all CTAs resident, one per SM) in which the ranges of each cut unit
   // wait for one another and share its rows, so a call is one launch.  It is the default for
   // decode and paged calls when every unit gets at least two ranges (the aligned split above)
-  // and a range holds at most 32 key tiles at the plan's context capacity: there the
+  // and a range holds at most 32 key tiles at the plan's (non-zero) context capacity: there the
   // combine's fixed cost is a large share of a short step (L = 4096: step 36.0 -> 33.3 us).
   // With long ranges the step gains little (L = 131072: 154.9 -> 153.5 us) while the
   // attention kernel's own time grows by the combine's work; with fewer ranges per unit
@@ -394,8 +394,9 @@ tt_status_t tt_block_attn_plan(const tt_block_attn_desc* desc, int device, tt_pl
     const bool can = P->kernel == TT_KERNEL_TCGEN05 && P->variant == 0 && P->C > 1 && P->C <= P->sm_count;
     P->fused_combine = can && force == 1;
     const long long unit_tiles = 1 + (long long)tt::ceil_div(d.ctx_capacity, P->key_tile);
-    const bool short_ranges =
-        decode_aligned && unit_tiles * d.batch * d.num_kv_heads <= 32LL * std::max(P->C_decode, 1);
+    // (a plan without a context capacity serves paged calls, whose lengths it cannot bound)
+    const bool short_ranges = decode_aligned && d.ctx_capacity > 0 &&
+                              unit_tiles * d.batch * d.num_kv_heads <= 32LL * std::max(P->C_decode, 1);
     P->fused_decode = can && P->C_decode <= P->sm_count && (force == 1 || (force != 0 && short_ranges));
   }
   P->causal_pref = pref.empty() ? nullptr : reinterpret_cast<int*>(w + b_po + b_pl + b_rec + b_err);
