@@ -131,7 +131,12 @@ TT_API tt_status_t tt_block_attn_plan_get_info(tt_plan_t plan, tt_plan_info* inf
  *   out      [B, S, Hq, D]    fp32  attention output
  *   lse      [B, Hq, S]       fp32  natural-log log-sum-exp per row; may be NULL
  * Context rows at or beyond L_n are never used, whatever they hold.  Out-of-range
- * ctx_lens values are clamped on the device and flagged TT_ERR_DEVICE_ARG. */
+ * ctx_lens values are clamped on the device and flagged TT_ERR_DEVICE_ARG.
+ * Launches, all on `stream`: the attention kernel, then (when units were cut over
+ * several work ranges) the split combine kernel, launched as its programmatic
+ * dependent.  Plans whose units all get at least two ranges, each of at most 32 key
+ * tiles at the plan's context capacity, launch the attention kernel cooperatively
+ * and combine in its tail instead: one launch per call (tt_plan_info.fused_combine). */
 TT_API tt_status_t tt_block_attn(tt_plan_t plan, const void* q, const void* k_ctx, const void* v_ctx,
                           const void* k_blk, const void* v_blk, const int32_t* ctx_lens,
                           float* out, float* lse, tt_stream_t stream);
@@ -283,7 +288,8 @@ TT_API tt_status_t tt_block_attn_check(tt_plan_t plan, tt_stream_t stream);
  * launches are kept).  tt_block_attn_profile_read synchronises on the recorded
  * events and returns, for kernel id 0 (attention), 1 (split combine) or 2
  * (block-causal backward), the number of launches and their summed duration in
- * milliseconds.  Calling
+ * milliseconds.  In a stream being captured into a CUDA graph the events are
+ * recorded as graph nodes, so the graph's replays are timed.  Calling
  * tt_block_attn_profile again clears the record. */
 TT_API tt_status_t tt_block_attn_profile(tt_plan_t plan, int enable);
 TT_API tt_status_t tt_block_attn_profile_read(tt_plan_t plan, int kernel_id, int* launches, double* total_ms);

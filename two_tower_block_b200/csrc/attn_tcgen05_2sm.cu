@@ -25,11 +25,11 @@
 // waits for that product only when O must be rescaled.  The two partial
 // softmax states of a row are merged exactly in the epilogue.
 //
-// The MMA thread issues S(j+2) interleaved, instruction by instruction, with P(j-1) V
+// The MMA warp issues S(j+2) interleaved, instruction by instruction, with P(j-1) V
 // (the other warpgroup's product), so that two independent accumulator chains are in
 // flight (the ring order below follows).
 //
-// Synchronisation across the pair: the even CTA's MMA thread commits with
+// Synchronisation across the pair: the even CTA's MMA warp commits with
 // multicast to barriers in both CTAs.  The odd CTA's TMA completions and softmax
 // arrivals land on its own barriers and are forwarded to the even CTA's by
 // otherwise idle warps (remote mbarrier arrive), so no softmax warp pays for a
