@@ -78,6 +78,8 @@ typedef enum {
 } tt_kernel_t;
 
 #define TT_PLAN_HOST_IO 1   /* flags: allocate device staging for tt_block_attn_host */
+#define TT_PLAN_OUT_BF16 2  /* flags: `out` of the decode, paged, host and block-causal calls is
+                               bf16 (round to nearest even) instead of fp32; lse stays fp32 */
 
 typedef struct {
   int batch;          /* B >= 0 (B = 0 makes every call a no-op)                    */
@@ -90,7 +92,7 @@ typedef struct {
   float scale;        /* softmax scale; 0 selects 1/sqrt(head_dim)                   */
   int kernel;         /* tt_kernel_t                                                 */
   int num_ctas;       /* persistent grid size; 0 selects the device's SM count       */
-  int flags;          /* TT_PLAN_HOST_IO or 0                                        */
+  int flags;          /* TT_PLAN_HOST_IO | TT_PLAN_OUT_BF16, or 0                    */
   int wait_timeout_us;/* limit of every in-kernel wait; 0 selects 1000000 (1 s)      */
 } tt_block_attn_desc;
 
@@ -128,7 +130,7 @@ TT_API tt_status_t tt_block_attn_plan_get_info(tt_plan_t plan, tt_plan_info* inf
  *   k_blk    [B, S, Hkv, D]   bf16  the denoiser's own block keys
  *   v_blk    [B, S, Hkv, D]   bf16  the denoiser's own block values
  *   ctx_lens [B]              int32 committed context length L_n, 0 <= L_n <= Lcap
- *   out      [B, S, Hq, D]    fp32  attention output
+ *   out      [B, S, Hq, D]    fp32  attention output (bf16 on a TT_PLAN_OUT_BF16 plan)
  *   lse      [B, Hq, S]       fp32  natural-log log-sum-exp per row; may be NULL
  * Context rows at or beyond L_n are never used, whatever they hold.  Out-of-range
  * ctx_lens values are clamped on the device and flagged TT_ERR_DEVICE_ARG.
@@ -176,7 +178,7 @@ TT_API tt_status_t tt_block_attn_paged(tt_plan_t plan, const void* q, const void
                                 tt_stream_t stream);
 
 /* Block-causal training / prefill form over whole sequences of length N = seq_len.
- *   q      [B, N, Hq, D]  bf16      out [B, N, Hq, D] fp32
+ *   q      [B, N, Hq, D]  bf16      out [B, N, Hq, D] fp32 (bf16 on a TT_PLAN_OUT_BF16 plan)
  *   k_ctx  [B, Hkv, N, D] bf16 (context tower over the clean sequence), v_ctx likewise
  *   k_blk  [B, N, Hkv, D] bf16 (denoiser over the noisy sequence),     v_blk likewise
  *   lse    [B, Hq, N] fp32 natural log, may be NULL
@@ -232,7 +234,8 @@ TT_API tt_status_t tt_block_attn_noalloc(const tt_block_attn_desc* desc, const v
  *   dq = scale sum_k ds k,  dk_blk[k] = scale sum_r ds q_r,  dv_blk[k] = sum_r p dout_r
  * (block keys only; summed over the g query heads of each KV head).
  *   q, k_ctx, v_ctx, k_blk, v_blk   the forward's inputs, layouts of tt_block_attn_block_causal
- *   out  [B, N, Hq, D] fp32, lse [B, Hq, N] fp32   the forward's outputs (lse required)
+ *   out  [B, N, Hq, D] fp32, lse [B, Hq, N] fp32   the forward's outputs (lse required);
+ *                                  a TT_PLAN_OUT_BF16 plan is rejected (TT_ERR_UNSUPPORTED)
  *   dout [B, N, Hq, D] bf16        dL/dout (a bf16 operand of the tensor cores, like q, k, v)
  *   dq   [B, N, Hq, D] fp32        written
  *   dk_blk, dv_blk [B, N, Hkv, D] fp32   cleared, then written

@@ -256,3 +256,26 @@ def test_binding_marshals_page_geometry_from_tensor_shapes(monkeypatch):
     assert a[5:8] == (7, 32, 5)                                   # num_pages, page_size, pages_per_seq
     assert a[1].value == q.data_ptr() and a[4].value == table.data_ptr() and a[10].value == lens.data_ptr()
     assert a[11].value == out.data_ptr() and a[12] is None        # no lse requested
+
+
+def test_binding_bf16_output_plan_wants_bf16_out():
+    """A plan made with out_bf16=True takes a bf16 `out` (2-byte elements) and rejects fp32."""
+    import torch
+    plan = _shape_only_plan()
+    plan.out_dtype = torch.bfloat16
+    B, S, Hq, Hkv, D, L = 2, 4, 8, 2, 64, 32
+    q = torch.zeros(B, S, Hq, D, dtype=torch.bfloat16)
+    kc = torch.zeros(B, Hkv, L, D, dtype=torch.bfloat16)
+    kb = torch.zeros(B, S, Hkv, D, dtype=torch.bfloat16)
+    lens = torch.zeros(B, dtype=torch.int32)
+    with pytest.raises(TypeError, match="out"):
+        plan.block_attn(q, kc, kc, kb, kb, lens, out=torch.zeros(B, S, Hq, D))
+    with pytest.raises(ValueError, match="cuda:0"):               # right dtype and size, host memory
+        plan.block_attn(q, kc, kc, kb, kb, lens, out=torch.zeros(B, S, Hq, D, dtype=torch.bfloat16))
+
+
+def test_plan_flag_values_match_the_header():
+    import re
+    hdr = open(os.path.join(os.path.dirname(__file__), "..", "include", "tt_block_attn.h")).read()
+    flags = {m.group(1): int(m.group(2)) for m in re.finditer(r"#define (TT_PLAN_\w+) (\d+)", hdr)}
+    assert flags == {"TT_PLAN_HOST_IO": ops.PLAN_HOST_IO, "TT_PLAN_OUT_BF16": ops.PLAN_OUT_BF16}

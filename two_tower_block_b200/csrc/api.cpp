@@ -170,6 +170,7 @@ tt::Problem base_problem(tt_plan_t plan) {
   p.wait_limit_ns = (unsigned long long)(d.wait_timeout_us > 0 ? d.wait_timeout_us : 1000000) * 1000ull;
   p.variant = plan->variant;
   p.arrivals = nullptr;
+  p.out_bf16 = (d.flags & TT_PLAN_OUT_BF16) ? 1 : 0;
   return p;
 }
 
@@ -267,7 +268,7 @@ tt_status_t tt_block_attn_plan(const tt_block_attn_desc* desc, int device, tt_pl
   if (!(d.scale >= 0.f) || std::isinf(d.scale)) return fail(TT_ERR_INVALID_ARG, "scale must be finite and >= 0");
   if (d.seq_len % d.block_size) return fail(TT_ERR_INVALID_ARG, "seq_len % block_size != 0");
   if (d.kernel < TT_KERNEL_AUTO || d.kernel > TT_KERNEL_MMA_SYNC) return fail(TT_ERR_INVALID_ARG, "unknown kernel");
-  if (d.flags & ~TT_PLAN_HOST_IO) return fail(TT_ERR_INVALID_ARG, "unknown flag bits");
+  if (d.flags & ~(TT_PLAN_HOST_IO | TT_PLAN_OUT_BF16)) return fail(TT_ERR_INVALID_ARG, "unknown flag bits");
   if (d.head_dim != 64 && d.head_dim != 128) return fail(TT_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
   const int g = d.num_q_heads / d.num_kv_heads;
   if ((long long)d.block_size * g > 256) return fail(TT_ERR_UNSUPPORTED, "block_size * (Hq/Hkv) must be <= 256");
@@ -310,6 +311,12 @@ tt_status_t tt_block_attn_plan(const tt_block_attn_desc* desc, int device, tt_pl
       if (tt::tcgen05_key_tile_supported(v)) P->key_tile = v;
     }
     if (P->variant == 3 && (!tt::attn_2sm_supported(d.head_dim, g) || P->key_tile != 128)) P->variant = 0;
+    // the bf16 output is written by the default kernel's epilogue (and the combine): the
+    // transposed-PV and 2-SM forms, selectable for fp32 output only, fall back to it
+    if ((d.flags & TT_PLAN_OUT_BF16) && P->variant != 0) {
+      P->variant = 0;
+      P->key_tile = tt::kTcgen05KeyTile;
+    }
     P->C = d.num_ctas > 0 ? d.num_ctas : P->sm_count;
     if (P->variant == 3) {
       // one range per cluster of two CTAs; by default as many as can be resident at once
@@ -416,7 +423,7 @@ tt_status_t tt_block_attn_plan(const tt_block_attn_desc* desc, int device, tt_pl
     P->st_kc = up(B * Hkv * (size_t)d.ctx_capacity * D * 2);
     P->st_kb = up(B * S * Hkv * D * 2);
     P->st_lens = up(B * 4);
-    P->st_out = up(B * S * Hq * D * 4);
+    P->st_out = up(B * S * Hq * D * ((d.flags & TT_PLAN_OUT_BF16) ? 2 : 4));
     P->st_lse = up(B * Hq * S * 4);
     const size_t tot = P->st_q + 2 * P->st_kc + 2 * P->st_kb + P->st_lens + P->st_out + P->st_lse;
     e = cudaMalloc(&P->stage, std::max<size_t>(tot, 256));
@@ -590,7 +597,7 @@ tt_status_t tt_block_attn_host(tt_plan_t plan, const void* q, const void* k_ctx,
                                 reinterpret_cast<const int32_t*>(dl), reinterpret_cast<float*>(dout),
                                 lse ? reinterpret_cast<float*>(dlse) : nullptr, stream);
   if (r != TT_OK) return r;
-  e = cudaMemcpyAsync(out, dout, B * S * Hq * D * 4, cudaMemcpyDeviceToHost, s);
+  e = cudaMemcpyAsync(out, dout, B * S * Hq * D * ((d.flags & TT_PLAN_OUT_BF16) ? 2 : 4), cudaMemcpyDeviceToHost, s);
   if (e == cudaSuccess && lse) e = cudaMemcpyAsync(lse, dlse, B * Hq * S * 4, cudaMemcpyDeviceToHost, s);
   if (e != cudaSuccess) return cuda_fail(e, "device-to-host copy");
   return TT_OK;
@@ -603,6 +610,8 @@ tt_status_t tt_block_attn_block_causal_backward(tt_plan_t plan, const void* q, c
   if (!plan) return fail(TT_ERR_INVALID_ARG, "null plan");
   const tt_block_attn_desc& d = plan->desc;
   if (d.seq_len == 0) return fail(TT_ERR_INVALID_ARG, "plan has seq_len == 0 (decode-only)");
+  if (d.flags & TT_PLAN_OUT_BF16)
+    return fail(TT_ERR_UNSUPPORTED, "the backward takes the fp32 forward output: use a plan without TT_PLAN_OUT_BF16");
   if (d.batch == 0) return TT_OK;
   if (!q || !k_ctx || !v_ctx || !k_blk || !v_blk || !out || !lse || !dout || !dq || !dk_blk || !dv_blk)
     return fail(TT_ERR_INVALID_ARG, "null tensor pointer");

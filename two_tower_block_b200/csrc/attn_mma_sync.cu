@@ -215,13 +215,13 @@ __global__ void __launch_bounds__(kThreads) attn_mma_sync_kernel(const Problem p
       const float inv = 1.f / l;
       const float lse = ((half ? m1 : m0) + __log2f(l)) * 0.6931471805599453f;
       const int t = r / p.g, j = r - (r / p.g) * p.g;
-      float* dst;
-      if (sg.full) dst = p.out + ((size_t)(x.ns * p.S + t) * p.Hq + x.h * p.g + j) * D;
-      else dst = p.part_o + ((size_t)sg.slot * p.R + r) * D;
+      const size_t off = out_offset(p, x, r, D);
+      float* part = p.part_o + ((size_t)sg.slot * p.R + r) * D;
 #pragma unroll
       for (int db = 0; db < D / 8; ++db) {
         float2 v = make_float2(o[db][2 * half] * inv, o[db][2 * half + 1] * inv);
-        *reinterpret_cast<float2*>(dst + db * 8 + 2 * qq) = v;
+        if (sg.full) store_out2(p, off + db * 8 + 2 * qq, v);
+        else *reinterpret_cast<float2*>(part + db * 8 + 2 * qq) = v;
       }
       if (qq == 0) {
         if (sg.full) {

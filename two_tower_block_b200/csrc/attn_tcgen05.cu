@@ -540,8 +540,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int gr = rbase + rr;
             if (gr < p.R) {
               float4 f = reinterpret_cast<const float4*>(stage + rr * 32)[q ^ (rr & 7)];
-              float* dst = out_row(p, x, sg, gr, D) + cc * 32 + q * 4;
-              *reinterpret_cast<float4*>(dst) = f;
+              if (sg.full) store_out4(p, out_offset(p, x, gr, D) + cc * 32 + q * 4, f);
+              else *reinterpret_cast<float4*>(out_row(p, x, sg, gr, D) + cc * 32 + q * 4) = f;
             }
           }
           __syncwarp();

@@ -75,11 +75,11 @@ __device__ __forceinline__ void combine_row(const Problem& p, int c, const Split
   }
   const float inv = 1.f / wsum;
   const int t = r / p.g, j = r - (r / p.g) * p.g;
-  float* dst = p.out + ((size_t)(x.ns * p.S + t) * p.Hq + x.h * p.g + j) * D + lane * V;
+  const size_t off = out_offset(p, x, r, D) + lane * V;
   if constexpr (V == 4) {
-    *reinterpret_cast<float4*>(dst) = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+    store_out4(p, off, make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv));
   } else {
-    *reinterpret_cast<float2*>(dst) = make_float2(acc[0] * inv, acc[1] * inv);
+    store_out2(p, off, make_float2(acc[0] * inv, acc[1] * inv));
   }
   if (lane == 0 && p.lse)
     p.lse[(size_t)(x.n * p.Hq + x.h * p.g + j) * (p.NB * p.S) + x.b * p.S + t] = M + logf(wsum);

@@ -33,8 +33,9 @@ struct Problem {
   const __nv_bfloat16* k_blk;
   const __nv_bfloat16* v_blk;
   const int* ctx_lens;  // decode only
-  float* out;
+  float* out;           // fp32, or bf16 when out_bf16 (the pointer then addresses bf16 elements)
   float* lse;           // may be null
+  int out_bf16;         // final output rows in bf16 (round to nearest even); partials stay fp32
   // work split
   int C;                // ranges
   int key_tile;         // keys per tile

@@ -155,6 +155,26 @@ __device__ __forceinline__ SplitRecord record_of(const Unit& last, long long T, 
   return r;
 }
 
+// Element offset of packed row r of unit x in the final output [.., S, Hq, D].
+__device__ __forceinline__ size_t out_offset(const Problem& p, const Unit& x, int r, int D) {
+  const int t = r / p.g, j = r - (r / p.g) * p.g;
+  return ((size_t)(x.ns * p.S + t) * p.Hq + x.h * p.g + j) * D;
+}
+// Four (or two) consecutive final-output values at element offset off: fp32, or bf16 pairs
+// rounded to nearest even when the problem asks for a bf16 output.
+__device__ __forceinline__ void store_out4(const Problem& p, size_t off, float4 v) {
+  if (p.out_bf16) {
+    const uint2 u = make_uint2(pack_bf16(v.x, v.y), pack_bf16(v.z, v.w));
+    *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(p.out) + off) = u;
+  } else {
+    *reinterpret_cast<float4*>(p.out + off) = v;
+  }
+}
+__device__ __forceinline__ void store_out2(const Problem& p, size_t off, float2 v) {
+  if (p.out_bf16) *reinterpret_cast<uint32_t*>(reinterpret_cast<__nv_bfloat16*>(p.out) + off) = pack_bf16(v.x, v.y);
+  else *reinterpret_cast<float2*>(p.out + off) = v;
+}
+
 // Keys of unit-local tile i: block keys for i < blk_tiles, context keys after.
 struct TileKeys {
   bool is_blk;

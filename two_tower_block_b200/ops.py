@@ -22,6 +22,7 @@ __all__ = ["TTError", "Plan", "lib", "library_path", "block_attn", "block_attn_b
 TT_OK, TT_ERR_INVALID_ARG, TT_ERR_UNSUPPORTED, TT_ERR_CUDA, TT_ERR_DEVICE_ARG, TT_ERR_TIMEOUT = range(6)
 KERNEL_AUTO, KERNEL_TCGEN05, KERNEL_MMA_SYNC = 0, 1, 2
 PLAN_HOST_IO = 1
+PLAN_OUT_BF16 = 2
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 library_path = os.path.join(_HERE, "libtt_block_attn.so")
@@ -165,14 +166,17 @@ class Shape:
 class Plan:
     """Owns a tt_plan_t (device scratch, work split) for one shape on one device."""
 
+    out_dtype = torch.float32   # torch.bfloat16 for a plan made with out_bf16=True
+
     def __init__(self, batch, q_heads, kv_heads, head_dim, block, ctx_capacity=0, seq_len=0, scale=0.0,
-                 kernel=KERNEL_AUTO, num_ctas=0, host_io=False, wait_timeout_us=0, device=None):
+                 kernel=KERNEL_AUTO, num_ctas=0, host_io=False, wait_timeout_us=0, device=None, out_bf16=False):
         if device is None:
             device = torch.cuda.current_device()
         self.shape = Shape(batch, q_heads, kv_heads, head_dim, block, ctx_capacity, seq_len)
         self.device = int(device)
+        self.out_dtype = torch.bfloat16 if out_bf16 else torch.float32
         d = Desc(batch, q_heads, kv_heads, head_dim, block, ctx_capacity, seq_len, float(scale), kernel,
-                 num_ctas, PLAN_HOST_IO if host_io else 0, wait_timeout_us)
+                 num_ctas, (PLAN_HOST_IO if host_io else 0) | (PLAN_OUT_BF16 if out_bf16 else 0), wait_timeout_us)
         h = ctypes.c_void_p()
         _check(lib().tt_block_attn_plan(ctypes.byref(d), self.device, ctypes.byref(h)), "tt_block_attn_plan")
         self._h = h
@@ -198,7 +202,7 @@ class Plan:
                    want_lse=False):
         s = self.shape
         if out is None:
-            out = torch.empty((s.batch, s.block, s.q_heads, s.head_dim), dtype=torch.float32, device=q.device)
+            out = torch.empty((s.batch, s.block, s.q_heads, s.head_dim), dtype=self.out_dtype, device=q.device)
         if lse is None and want_lse:
             lse = torch.empty((s.batch, s.q_heads, s.block), dtype=torch.float32, device=q.device)
         nc = s.batch * s.kv_heads * s.ctx_capacity * s.head_dim
@@ -213,8 +217,11 @@ class Plan:
         nq = s.batch * s.block * s.q_heads * s.head_dim
         nb = s.batch * s.block * s.kv_heads * s.head_dim
         return [(q, "q", nq, "bf16"), (k_blk, "k_blk", nb, "bf16"), (v_blk, "v_blk", nb, "bf16"),
-                (ctx_lens, "ctx_lens", s.batch, "i32"), (out, "out", nq, "f32"),
+                (ctx_lens, "ctx_lens", s.batch, "i32"), (out, "out", nq, self._out_kind()),
                 (lse, "lse", s.batch * s.q_heads * s.block, "f32")]
+
+    def _out_kind(self):
+        return "bf16" if self.out_dtype == torch.bfloat16 else "f32"
 
     def block_attn_paged(self, q, k_pages, v_pages, page_table, k_blk, v_blk, ctx_lens, out=None, lse=None,
                          stream=None, want_lse=False):
@@ -223,7 +230,7 @@ class Plan:
         context at all, the pools and the table may be None."""
         s = self.shape
         if out is None:
-            out = torch.empty((s.batch, s.block, s.q_heads, s.head_dim), dtype=torch.float32, device=q.device)
+            out = torch.empty((s.batch, s.block, s.q_heads, s.head_dim), dtype=self.out_dtype, device=q.device)
         if lse is None and want_lse:
             lse = torch.empty((s.batch, s.q_heads, s.block), dtype=torch.float32, device=q.device)
         if k_pages is None:
@@ -264,21 +271,21 @@ class Plan:
                                 want_lse=False):
         s = self.shape
         if out is None:
-            out = torch.empty((s.batch, s.seq_len, s.q_heads, s.head_dim), dtype=torch.float32, device=q.device)
+            out = torch.empty((s.batch, s.seq_len, s.q_heads, s.head_dim), dtype=self.out_dtype, device=q.device)
         if lse is None and want_lse:
             lse = torch.empty((s.batch, s.q_heads, s.seq_len), dtype=torch.float32, device=q.device)
-        _args(self.device, *self._causal_items(q, k_ctx, v_ctx, k_blk, v_blk, out, lse))
+        _args(self.device, *self._causal_items(q, k_ctx, v_ctx, k_blk, v_blk, out, lse, self._out_kind()))
         _check(lib().tt_block_attn_block_causal(self._h, _ptr(q), _ptr(k_ctx), _ptr(v_ctx), _ptr(k_blk),
                                                 _ptr(v_blk), _ptr(out), _ptr(lse), _stream(stream)),
                "tt_block_attn_block_causal")
         return (out, lse) if want_lse or lse is not None else out
 
-    def _causal_items(self, q, k_ctx, v_ctx, k_blk, v_blk, out, lse):
+    def _causal_items(self, q, k_ctx, v_ctx, k_blk, v_blk, out, lse, out_kind="f32"):
         s = self.shape
         nq = s.batch * s.seq_len * s.q_heads * s.head_dim
         nk = s.batch * s.seq_len * s.kv_heads * s.head_dim
         return [(q, "q", nq, "bf16"), (k_ctx, "k_ctx", nk, "bf16"), (v_ctx, "v_ctx", nk, "bf16"),
-                (k_blk, "k_blk", nk, "bf16"), (v_blk, "v_blk", nk, "bf16"), (out, "out", nq, "f32"),
+                (k_blk, "k_blk", nk, "bf16"), (v_blk, "v_blk", nk, "bf16"), (out, "out", nq, out_kind),
                 (lse, "lse", s.batch * s.q_heads * s.seq_len, "f32")]
 
     def block_causal_backward(self, q, k_ctx, v_ctx, k_blk, v_blk, out, lse, dout, dq=None, dk_blk=None,
