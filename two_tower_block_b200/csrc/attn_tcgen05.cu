@@ -207,6 +207,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(smem_u32(&sh->tmem_base), 512);
     tmem_relinquish();
   }
+  // launched as a programmatic dependent of the previous kernel on the stream: everything above
+  // (barriers, TMEM, descriptor prefetch) overlaps that kernel's tail; nothing below reads or
+  // writes global memory before it has completed
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   if (warp == 2) {
     long long T = 0, start = 0, end = 0;
     Unit first;
@@ -591,21 +595,20 @@ void set_smem_attr() {
 
 template <int D, int NK>
 cudaError_t launch(const Problem& p, const TmaMaps& maps, cudaStream_t stream) {
-  if (p.arrivals == nullptr) {
-    attn_tcgen05_kernel<D, NK><<<p.C, kThreads, Cfg<D, NK>::kSmemBytes, stream>>>(p, maps);
-    return cudaGetLastError();
-  }
-  // cooperative: every CTA must be resident at once for the waits of the fused combine
+  // a programmatic dependent of the previous kernel on the stream (its setup overlaps that
+  // kernel's tail), and cooperative when the fused combine needs every CTA resident at once
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.C, 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = Cfg<D, NK>::kSmemBytes;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeCooperative;
-  attr[0].val.cooperative = 1;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeCooperative;
+  attr[1].val.cooperative = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = p.arrivals != nullptr ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, attn_tcgen05_kernel<D, NK>, p, maps);
 }
 

@@ -14,7 +14,9 @@ constexpr int kThreads = 256;
 template <int D>
 __global__ void __launch_bounds__(kThreads) combine_kernel(const Problem p) {
   // launched as a programmatic dependent of the attention kernel: wait until its grid has
-  // completed and its partials are visible
+  // completed and its partials are visible; the next call's attention kernel may be scheduled
+  // meanwhile and waits for this grid itself
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int c = blockIdx.x;
   const SplitRecord rec = p.records[c];
