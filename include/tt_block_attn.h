@@ -183,7 +183,13 @@ TT_API tt_status_t tt_block_attn_paged(tt_plan_t plan, const void* q, const void
  *   k_blk  [B, N, Hkv, D] bf16 (denoiser over the noisy sequence),     v_blk likewise
  *   lse    [B, Hq, N] fp32 natural log, may be NULL
  * Block b = positions [S*b, S*b+S) attends to k_ctx positions [0, S*b) and to its
- * own k_blk positions, bidirectionally.  Requires a plan with seq_len > 0. */
+ * own k_blk positions, bidirectionally.  Requires a plan with seq_len > 0.
+ * Work split: the B*Hkv*(N/S) units (one per block and KV head) are laid end to end
+ * in key tiles and cut into the plan's ranges.  On the default tcgen05 kernel the
+ * boundaries weigh each unit as its key tiles plus a fixed cost of 8 tiles (its Q
+ * load and pipeline restart, and its output epilogue), so that ranges of many short
+ * early blocks take no longer than ranges of a few long late ones; the other kernels
+ * split the tiles evenly.  tt_debug_causal_split shows the boundaries. */
 TT_API tt_status_t tt_block_attn_block_causal(tt_plan_t plan, const void* q, const void* k_ctx,
                                        const void* v_ctx, const void* k_blk, const void* v_blk,
                                        float* out, float* lse, tt_stream_t stream);
@@ -319,6 +325,19 @@ TT_API tt_status_t tt_selftest_exp2(int device, const float* x, float* y, int n)
  * code decides the split inside the kernels. */
 TT_API tt_status_t tt_debug_work_split(int num_units, const int* tiles_per_unit, int num_ctas,
                                 long long* range_start, int* unit_first, int* unit_last);
+
+/* Host-only view of the block-causal work split of the default tcgen05 kernel (no
+ * GPU needed): for B = batch sequences of seq_len positions in blocks of
+ * block_size, Hkv = num_kv_heads and key_tile keys per tile, writes the first
+ * global tile of each of the num_ctas ranges and the total T (range_start, host,
+ * num_ctas + 1 entries; ranges beyond min(num_ctas, T) start at T).  unit_cost is
+ * the fixed cost of a unit in key tiles: -1 takes the plan's default (8), 0 gives
+ * the even split of tt_debug_work_split.  The plan builds its table with the same
+ * code.  TT_ERR_INVALID_ARG for non-positive sizes, seq_len not a multiple of
+ * block_size or a NULL range_start; TT_ERR_UNSUPPORTED when one (n, h) has 2^31
+ * tiles or more. */
+TT_API tt_status_t tt_debug_causal_split(int batch, int num_kv_heads, int seq_len, int block_size,
+                                         int key_tile, int num_ctas, int unit_cost, long long* range_start);
 
 TT_API const char* tt_status_string(tt_status_t status);
 

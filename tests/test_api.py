@@ -122,6 +122,65 @@ def test_work_split_partition(tiles, C):
     assert len(cut_starts) == len(set(cut_starts))
 
 
+def _causal_tiles(B, Hkv, N, S, kt):
+    """Key tiles of each block-causal unit in the kernel's order ((n, h) major, block b minor):
+    the block's own S keys, then its S*b context keys, key_tile at a time."""
+    one = [-(-S // kt) + -(-S * b // kt) for b in range(N // S)]
+    return one * (B * Hkv)
+
+
+def _modelled_range_times(tiles, starts, unit_cost):
+    """Per range: its tiles plus unit_cost for every unit it touches (a cut unit counts in each
+    range that holds a piece of it: each piece loads Q and writes an epilogue)."""
+    Tu = np.concatenate([[0], np.cumsum(tiles)])
+    out = []
+    for c in range(len(starts) - 1):
+        s, e = starts[c], starts[c + 1]
+        if e <= s:
+            continue
+        u0 = np.searchsorted(Tu, s, side="right") - 1
+        u1 = np.searchsorted(Tu, e, side="left")
+        out.append((e - s) + unit_cost * (u1 - u0))
+    return np.array(out, dtype=np.float64)
+
+
+@pytest.mark.parametrize("B,Hkv,N,S,kt,C", [
+    (8, 2, 8192, 16, 64, 148), (1, 2, 8192, 16, 64, 148), (2, 4, 4096, 32, 64, 148), (1, 1, 2048, 16, 128, 37),
+    (3, 2, 1024, 16, 64, 148), (1, 1, 64, 16, 64, 148), (1, 1, 16, 16, 64, 148), (1, 1, 256, 16, 64, 1),
+])
+def test_causal_split_weighs_units(B, Hkv, N, S, kt, C):
+    """The block-causal boundaries partition [0, T) into min(C, T) non-empty ranges; with no
+    unit cost they are the even split; with the default cost the modelled range times (tiles +
+    8 per touched unit) are balanced far better than the even split's, which puts the many
+    short early blocks of each (n, h) into a few ranges."""
+    tiles = _causal_tiles(B, Hkv, N, S, kt)
+    T = sum(tiles)
+    Ce = min(C, T)
+    even = ops.causal_split(B, Hkv, N, S, kt, C, 0)
+    assert even == ops.work_split(tiles, C)[0]
+    starts = ops.causal_split(B, Hkv, N, S, kt, C)
+    assert starts[0] == 0 and starts[Ce] == T and all(x == T for x in starts[Ce:])
+    assert all(starts[c] < starts[c + 1] for c in range(Ce))
+    if T <= C:
+        assert starts == even   # one tile per range: nothing to weigh
+        return
+    w = _modelled_range_times(tiles, starts, 8)
+    e = _modelled_range_times(tiles, even, 8)
+    # a boundary moves by at most one unit's fixed cost to stay off it: within one unit cost
+    # of the mean (the even split is off by 1.6 to 2.1 x the mean on these shapes)
+    assert w.max() - w.mean() <= 8 + 1
+    assert w.max() <= e.max()
+    if (B, N) == (1, 8192):
+        assert e.max() / e.mean() > 1.6 and w.max() / w.mean() < 1.02
+
+
+def test_causal_split_rejects_bad_geometry():
+    for args in [(0, 1, 64, 16, 64, 4), (1, 1, 60, 16, 64, 4), (1, 1, 64, 16, 0, 4), (1, 1, 64, 16, 64, 0),
+                 (1, 0, 64, 16, 64, 4), (1, 1, 8, 16, 64, 4)]:
+        with pytest.raises(RuntimeError):
+            ops.causal_split(*args)
+
+
 def test_no_device_plan_creation_reports_cuda_error():
     """Without a visible GPU a valid descriptor yields TT_ERR_CUDA (never a CPU path)."""
     import torch

@@ -106,6 +106,7 @@ struct tt_plan_s {
   bool fused_decode = false;    // decode and paged calls do
   int* causal_pref = nullptr;
   long long causal_T = 0;
+  long long* causal_starts = nullptr;   // weighted range boundaries of block-causal calls, or null
   int causal_NB = 0;
   // host IO staging
   void* stage = nullptr;
@@ -237,6 +238,64 @@ tt_status_t launch_all(tt_plan_t plan, const tt::Problem& p, cudaStream_t s) {
     if (e != cudaSuccess) return cuda_fail(e, "combine kernel launch");
   }
   return TT_OK;
+}
+
+// Range boundaries of the block-causal calls of the default tcgen05 kernel, weighted so that
+// every range carries the same modelled time: a unit costs its key tiles plus a fixed cost of
+// kCausalUnitCost tiles, half before its first tile (the Q load and the pipeline's restart) and
+// half after its last (the output epilogue).  The boundaries split that weighted sequence
+// evenly; one that falls in a unit's fixed cost moves to the unit's edge (no cut), one that
+// falls among its tiles cuts the unit there.  With the uniform split the first ranges of each
+// (n, h), which hold many short units, ran up to 1.7 x the mean range's time; a fixed cost of
+// about 8 tiles per unit of two M-tiles reproduces that spread.  TT_CAUSAL_UNIT_COST overrides
+// the cost (0: the uniform split, no table).
+constexpr int kCausalUnitCost = 8;
+
+// The table for `pairs` (n, h) pairs of NB units each, pref the tile prefix over b (NB + 1
+// entries), C ranges and a unit cost of H tiles: min(C, T) + 1 entries, or none when the
+// uniform split applies (H = 0 or a single range).
+std::vector<long long> weighted_causal_starts(const std::vector<int>& pref, long long pairs, int C, long long H) {
+  std::vector<long long> tab;
+  if (pref.size() < 2 || pairs <= 0) return tab;
+  const int NB = (int)pref.size() - 1;
+  const long long T = pairs * pref[NB];
+  const int Ce = tt::used_ranges(T, C);
+  if (H <= 0 || Ce <= 1) return tab;
+  const long long U = pairs * NB;
+  const long long H0 = H / 2;          // weight before a unit's first tile
+  const long long V = T + H * U;       // weighted length
+  tab.assign(Ce + 1, 0);
+  tab[Ce] = T;
+  long long u = 0, vbase = 0, base = 0;  // unit, its weighted and its tile offset
+  for (int c = 1; c < Ce; ++c) {
+    const long long v = (long long)((__int128)c * V / Ce);
+    for (; u < U; ++u) {
+      const int b = (int)(u % NB);
+      const long long t = pref[b + 1] - pref[b];
+      if (vbase + t + H > v) break;
+      vbase += t + H;
+      base += t;
+    }
+    if (u >= U) {
+      tab[c] = T;
+    } else {
+      const int b = (int)(u % NB);
+      const long long t = pref[b + 1] - pref[b];
+      tab[c] = base + std::min(std::max(v - vbase - H0, 0LL), t);
+    }
+  }
+  // strictly increasing: every range holds at least one tile
+  for (int c = 1; c < Ce; ++c) tab[c] = std::max(tab[c], tab[c - 1] + 1);
+  for (int c = Ce - 1; c >= 1; --c) tab[c] = std::min(tab[c], tab[c + 1] - 1);
+  return tab;
+}
+
+std::vector<long long> causal_range_table(const tt_plan_s* P, const std::vector<int>& pref,
+                                          const tt_block_attn_desc& d) {
+  if (pref.empty() || P->kernel != TT_KERNEL_TCGEN05 || P->variant != 0) return {};
+  long long H = kCausalUnitCost;
+  if (const char* s = std::getenv("TT_CAUSAL_UNIT_COST")) H = std::max(0, std::atoi(s));
+  return weighted_causal_starts(pref, (long long)d.batch * d.num_kv_heads, P->C, H);
 }
 
 }  // namespace
@@ -372,7 +431,9 @@ tt_status_t tt_block_attn_plan(const tt_block_attn_desc* desc, int device, tt_pl
   const size_t b_err = 256;
   const size_t b_pref = up(pref.size() * sizeof(int));
   const size_t b_arr = up((size_t)2 * Cmax * sizeof(unsigned));
-  P->ws_bytes = b_po + b_pl + b_rec + b_err + b_pref + b_arr;
+  const std::vector<long long> tab = causal_range_table(P, pref, d);
+  const size_t b_tab = up(tab.size() * sizeof(long long));
+  P->ws_bytes = b_po + b_pl + b_rec + b_err + b_pref + b_arr + b_tab;
   e = cudaMalloc(&P->ws, P->ws_bytes);
   if (e != cudaSuccess) {
     delete P;
@@ -407,10 +468,13 @@ tt_status_t tt_block_attn_plan(const tt_block_attn_desc* desc, int device, tt_pl
     P->fused_decode = can && P->C_decode <= P->sm_count && (force == 1 || (force != 0 && short_ranges));
   }
   P->causal_pref = pref.empty() ? nullptr : reinterpret_cast<int*>(w + b_po + b_pl + b_rec + b_err);
+  P->causal_starts = tab.empty() ? nullptr : reinterpret_cast<long long*>(w + b_po + b_pl + b_rec + b_err + b_pref + b_arr);
   e = cudaMemset(P->err_word, 0, b_err);
   if (e == cudaSuccess) e = cudaMemset(P->arr_decode, 0, b_arr);
   if (e == cudaSuccess && !pref.empty())
     e = cudaMemcpy(P->causal_pref, pref.data(), pref.size() * sizeof(int), cudaMemcpyHostToDevice);
+  if (e == cudaSuccess && !tab.empty())
+    e = cudaMemcpy(P->causal_starts, tab.data(), tab.size() * sizeof(long long), cudaMemcpyHostToDevice);
   if (e != cudaSuccess) {
     cudaFree(P->ws);
     delete P;
@@ -559,6 +623,7 @@ tt_status_t tt_block_attn_block_causal(tt_plan_t plan, const void* q, const void
   p.lse = lse;
   p.T_causal = plan->causal_T;
   p.causal_pref = plan->causal_pref;
+  p.causal_starts = plan->causal_starts;
   return launch_all(plan, p, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -820,6 +885,28 @@ tt_status_t tt_debug_work_split(int num_units, const int* tiles_per_unit, int nu
     unit_last[u] = tt::range_of_tile(T, Ce, Tu + tiles_per_unit[u] - 1);
     Tu += tiles_per_unit[u];
   }
+  return TT_OK;
+}
+
+tt_status_t tt_debug_causal_split(int batch, int num_kv_heads, int seq_len, int block_size, int key_tile,
+                                  int num_ctas, int unit_cost, long long* range_start) {
+  if (batch < 1 || num_kv_heads < 1 || block_size < 1 || seq_len < block_size || seq_len % block_size != 0 ||
+      key_tile < 1 || num_ctas < 1 || !range_start)
+    return fail(TT_ERR_INVALID_ARG, "bad arguments");
+  const int NB = seq_len / block_size;
+  std::vector<int> pref(NB + 1);
+  long long acc = 0;
+  for (int b = 0; b <= NB; ++b) {
+    pref[b] = (int)acc;
+    if (b < NB) acc += tt::ceil_div(block_size, key_tile) + tt::ceil_div(block_size * b, key_tile);
+    if (acc > (1ll << 31) - 1) return fail(TT_ERR_UNSUPPORTED, "sequence too long");
+  }
+  const long long T = (long long)batch * num_kv_heads * acc;
+  const std::vector<long long> tab =
+      weighted_causal_starts(pref, (long long)batch * num_kv_heads, num_ctas, unit_cost < 0 ? kCausalUnitCost : unit_cost);
+  const int Ce = tt::used_ranges(T, num_ctas);
+  for (int c = 0; c <= num_ctas; ++c)
+    range_start[c] = c > Ce ? T : tab.empty() ? tt::range_start(T, Ce, c) : tab[c];
   return TT_OK;
 }
 

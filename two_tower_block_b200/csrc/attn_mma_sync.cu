@@ -234,7 +234,7 @@ __global__ void __launch_bounds__(kThreads) attn_mma_sync_kernel(const Problem p
     }
 
     if (sg.last) {
-      if (rb == 0 && tid == 0) p.records[c] = record_of(x, T, p.C, start, end);
+      if (rb == 0 && tid == 0) p.records[c] = record_of(x, T, p.C, start, end, range_table(p));
       break;
     }
     x = make_unit(p, x.u + 1, x.Tu + x.tiles);

@@ -119,7 +119,8 @@ __device__ __forceinline__ void fused_combine(const Problem& p, long long T, lon
     const Unit x = which == 0 ? first : last;
     if (which == 1 && last.u == first.u) break;
     if (x.Tu >= start && x.Tu + x.tiles <= end) continue;  // whole in this range: not cut
-    const int c0 = range_of_tile(T, Ce, x.Tu), c1 = range_of_tile(T, Ce, x.Tu + x.tiles - 1);
+    const long long* tab = range_table(p);
+    const int c0 = range_of_tile_tab(tab, T, Ce, x.Tu), c1 = range_of_tile_tab(tab, T, Ce, x.Tu + x.tiles - 1);
     if (warp == 0) {
       bool ok = true;
       const unsigned long long t0 = globaltimer_ns();
@@ -139,7 +140,7 @@ __device__ __forceinline__ void fused_combine(const Problem& p, long long T, lon
     __syncthreads();
     if (!s_ok) return;
     const int n = c1 - c0 + 1, i = c - c0;
-    const SplitRecord rec{x.u, c1, x.Tu == range_start(T, Ce, c0) ? 0 : 1, 0};
+    const SplitRecord rec{x.u, c1, x.Tu == range_start_tab(tab, T, Ce, c0) ? 0 : 1, 0};
     const int r0 = (int)((long long)i * p.R / n), r1 = (int)((long long)(i + 1) * p.R / n);
     for (int r = r0 + warp; r < r1; r += kThreads / 32) combine_row<D, 16>(p, c0, rec, r, lane);
   }
@@ -574,7 +575,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (have_work) {
       Unit x = sh->first;
       while (x.Tu + x.tiles < end) x = make_unit(p, x.u + 1, x.Tu + x.tiles);
-      rec = record_of(x, T, p.C, start, end);
+      rec = record_of(x, T, p.C, start, end, range_table(p));
     }
     p.records[c] = rec;
   }

@@ -462,7 +462,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (have_work) {
       Unit x = ms->first;
       while (x.Tu + x.tiles < end) x = make_unit(p, x.u + 1, x.Tu + x.tiles);
-      rec = record_of(x, T, p.C, start, end);
+      rec = record_of(x, T, p.C, start, end, range_table(p));
     }
     p.records[c] = rec;
   }

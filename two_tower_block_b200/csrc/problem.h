@@ -42,6 +42,8 @@ struct Problem {
   int blk_tiles;        // tiles holding the block's own keys: ceil(S / key_tile)
   long long T_causal;   // block-causal: total tiles (decode computes T on the device)
   const int* causal_pref;  // block-causal: tiles before block b within one (n, h); NB + 1 entries
+  const long long* causal_starts;  // block-causal: range boundary table (min(C, T) + 1 entries) or
+                                   // null for the uniform split
   // plan-owned scratch
   float* part_o;        // [2C][R][D]
   float* part_lse;      // [2C][R]

@@ -15,6 +15,11 @@
 // range's first tile and 1 otherwise; a cut unit is then finished by the
 // combine kernel.  Only a range's first and last segment can belong to a cut
 // unit, so 2*C slots always suffice.
+//
+// A plan may instead give the boundaries as a table starts[0..C'] (starts[0] = 0,
+// starts[C'] = T, strictly increasing), which the block-causal calls of the default
+// kernel use to weigh each unit's fixed cost (built by the plan on the host); everything
+// above holds for it unchanged.
 #pragma once
 #include <stdint.h>
 
@@ -36,6 +41,21 @@ TT_HD int used_ranges(long long T, int C) { return T < (long long)C ? (int)T : C
 // the largest c with floor(c*T/C) <= x, i.e. ceil((x+1)*C/T) - 1.
 TT_HD int range_of_tile(long long T, int C, long long x) {
   return (int)(((x + 1) * (long long)C + T - 1) / T) - 1;
+}
+
+// The same two for a boundary table (null: the uniform split).
+TT_HD long long range_start_tab(const long long* tab, long long T, int C, int c) {
+  return tab ? tab[c] : range_start(T, C, c);
+}
+TT_HD int range_of_tile_tab(const long long* tab, long long T, int C, long long x) {
+  if (!tab) return range_of_tile(T, C, x);
+  int lo = 0, hi = C - 1;  // the largest c with tab[c] <= x
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (tab[mid] <= x) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo;
 }
 
 TT_HD int ceil_div(int a, int b) { return (a + b - 1) / b; }

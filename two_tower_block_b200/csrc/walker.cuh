@@ -55,6 +55,11 @@ __device__ __forceinline__ long long warp_sum_ll(long long v) {
   return v;
 }
 
+// The boundary table of the call's split, or null for the uniform one.
+__device__ __forceinline__ const long long* range_table(const Problem& p) {
+  return p.mode == kDecode ? nullptr : p.causal_starts;
+}
+
 // Called by one full warp.  Finds the total tile count T, this range's
 // [start, end) and the unit containing `start` (valid only if start < end).
 __device__ __forceinline__ void find_range(const Problem& p, int c, long long& T, long long& start,
@@ -77,8 +82,9 @@ __device__ __forceinline__ void find_range(const Problem& p, int c, long long& T
     start = end = T;
     return;
   }
-  start = range_start(T, Ce, c);
-  end = range_start(T, Ce, c + 1);
+  const long long* tab = range_table(p);
+  start = range_start_tab(tab, T, Ce, c);
+  end = range_start_tab(tab, T, Ce, c + 1);
   if (p.mode == kDecode) {
     long long acc = 0;
     for (int base = 0; base < p.B; base += 32) {
@@ -140,7 +146,7 @@ __device__ __forceinline__ Segment segment_of(const Unit& x, long long start, lo
 // The record of range c: the cut unit that begins in c and runs past its end.
 // C is the plan's range count; the split uses min(C, T) of them.
 __device__ __forceinline__ SplitRecord record_of(const Unit& last, long long T, int C, long long start,
-                                                 long long end) {
+                                                 long long end, const long long* tab) {
   C = used_ranges(T, C);
   SplitRecord r;
   r.unit = -1;
@@ -149,7 +155,7 @@ __device__ __forceinline__ SplitRecord record_of(const Unit& last, long long T, 
   r.pad = 0;
   if (last.Tu >= start && last.Tu + last.tiles > end) {
     r.unit = last.u;
-    r.last_range = range_of_tile(T, C, last.Tu + last.tiles - 1);
+    r.last_range = range_of_tile_tab(tab, T, C, last.Tu + last.tiles - 1);
     r.first_which = (last.Tu == start) ? 0 : 1;
   }
   return r;

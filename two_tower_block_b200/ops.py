@@ -34,6 +34,7 @@ EXPORTED_SYMBOLS = [
     "tt_block_attn_profile_read", "tt_selftest_wait_timeout", "tt_debug_work_split", "tt_status_string",
     "tt_last_error_detail", "tt_block_attn_noalloc", "tt_selftest_exp2", "tt_kv_append",
     "tt_block_attn_block_causal_backward", "tt_confidence_unmask", "tt_block_attn_paged",
+    "tt_debug_causal_split",
 ]
 
 
@@ -75,6 +76,7 @@ def lib() -> ctypes.CDLL:
     L.tt_block_attn_profile_read.argtypes = [vp, i, ip, ctypes.POINTER(ctypes.c_double)]
     L.tt_selftest_wait_timeout.argtypes = [i, i, vp]
     L.tt_debug_work_split.argtypes = [i, ip, i, ctypes.POINTER(ctypes.c_longlong), ip, ip]
+    L.tt_debug_causal_split.argtypes = [i, i, i, i, i, i, i, ctypes.POINTER(ctypes.c_longlong)]
     L.tt_block_attn_noalloc.argtypes = [ctypes.POINTER(Desc)] + [vp] * 10
     L.tt_selftest_exp2.argtypes = [i, vp, vp, i]
     L.tt_status_string.argtypes = [i]
@@ -416,6 +418,15 @@ def work_split(tiles_per_unit, num_ctas):
     last = (ctypes.c_int * max(n, 1))()
     _check(lib().tt_debug_work_split(n, tiles, num_ctas, starts, first, last), "tt_debug_work_split")
     return list(starts), list(first)[:n], list(last)[:n]
+
+
+def causal_split(batch, num_kv_heads, seq_len, block_size, key_tile, num_ctas, unit_cost=-1):
+    """Host-only: the range boundaries of a block-causal call on the default tcgen05 kernel
+    (unit_cost -1: the library's default fixed cost per unit; 0: the even split)."""
+    starts = (ctypes.c_longlong * (num_ctas + 1))()
+    _check(lib().tt_debug_causal_split(batch, num_kv_heads, seq_len, block_size, key_tile, num_ctas, unit_cost,
+                                       starts), "tt_debug_causal_split")
+    return list(starts)
 
 
 def block_attn_noalloc(q, k_ctx, v_ctx, k_blk, v_blk, ctx_lens, out, lse=None, status=None, scale=0.0,
