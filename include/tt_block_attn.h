@@ -138,7 +138,10 @@ TT_API tt_status_t tt_block_attn_plan_get_info(tt_plan_t plan, tt_plan_info* inf
  * several work ranges) the split combine kernel, launched as its programmatic
  * dependent.  Plans whose units all get at least two ranges, each of at most 32 key
  * tiles at the plan's context capacity, launch the attention kernel cooperatively
- * and combine in its tail instead: one launch per call (tt_plan_info.fused_combine). */
+ * and combine in its tail instead: one launch per call (tt_plan_info.fused_combine).
+ * The attention kernel is itself a programmatic dependent of the kernel before it on
+ * `stream`: its setup may overlap that kernel's tail, and it touches no global memory
+ * before that kernel has completed, so stream order holds as for a plain launch. */
 TT_API tt_status_t tt_block_attn(tt_plan_t plan, const void* q, const void* k_ctx, const void* v_ctx,
                           const void* k_blk, const void* v_blk, const int32_t* ctx_lens,
                           float* out, float* lse, tt_stream_t stream);
