@@ -161,6 +161,16 @@ def test_causal_split_weighs_units(B, Hkv, N, S, kt, C):
     starts = ops.causal_split(B, Hkv, N, S, kt, C)
     assert starts[0] == 0 and starts[Ce] == T and all(x == T for x in starts[Ce:])
     assert all(starts[c] < starts[c + 1] for c in range(Ce))
+    # the partial-slot bound of the split holds for the table too: at most one cut unit begins in
+    # any range (brute force over the units)
+    Tu = np.concatenate([[0], np.cumsum(tiles)])
+    cut_first = []
+    for u in range(len(tiles)):
+        touching = [c for c in range(Ce) if starts[c] < Tu[u + 1] and starts[c + 1] > Tu[u]]
+        assert touching == list(range(touching[0], touching[-1] + 1))
+        if len(touching) > 1:
+            cut_first.append(touching[0])
+    assert len(cut_first) == len(set(cut_first))
     if T <= C:
         assert starts == even   # one tile per range: nothing to weigh
         return
